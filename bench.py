@@ -1,0 +1,550 @@
+#!/usr/bin/env python
+"""Benchmark of the block-scaled microscaling hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the MXFP4 routed-expert workload: quantize bf16
+weights [8, 2048, 7168] to packed e2m1 + e8m0 scales, dequantize packed
+weights back to bf16 and to fp32 (three kernels).  Inputs (235 MB) and outputs
+are larger than the 126 MB L2, and the dequantize kernels read packed buffers
+written two steps earlier (three rotating slots), so every byte is an HBM byte.
+`value` is algorithmic bytes (each input read once, each output written once)
+per second over the timed region, summed over ranks (weak scaling: each rank
+runs its own copy of the workload; the path has no data exchange).
+
+The same run also times the other workloads as sub-measurements ("extra"):
+NVFP4 [256, 2048] round trip latency, the cache fake-quant cases, the
+[7168, 18432] NVFP4 weight quantization (ModelOpt per-tensor, per-row,
+gate/up) and the fused-dequant grouped GEMM (TFLOP/s), each with its HBM or
+tensor roofline.
+
+--impl reference times the CPU oracle (the only reference this path has) on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quant/dequant GB/s (% HBM peak); dequant grouped-GEMM TFLOP/s (% bf16 peak)"
+E, N, K = 8, 2048, 7168
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="skip the sub-measurements of the other workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--only", default="", help="comma list of extra sections to run (nvfp4,cache,linear,gemm)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fp8_microscaling_quantization_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles(kernel_key):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None
+    if the summary is missing or was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    ent = d.get("kernels", {}).get(kernel_key)
+    if not ent:
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        def reader():
+            for line in self.proc.stdout:
+                self.samples.append((time.time(), [s.strip() for s in line.split(",")]))
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        if self.proc is None:
+            return {"unavailable": "nvidia-smi not runnable"}
+        sel = [s for t, s in self.samples if t0 <= t <= t1 and len(s) >= 9]
+        if not sel:
+            sel = [s for t, s in self.samples if len(s) >= 9][-5:]
+        if not sel:
+            return {"unavailable": "no samples"}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = sorted(v for v in (num(s[1]) for s in sel) if v is not None)
+        mx = max((v for v in (num(s[2]) for s in sel) if v is not None), default=None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in sel for i in range(4) if s[5 + i].lower().startswith("active")})
+        pw = [v for v in (num(s[3]) for s in sel) if v is not None]
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(sel), "power_w_max": max(pw) if pw else None}
+
+
+# ------------------------------------------------------------------- utils --
+
+def mx_bytes():
+    n = E * N * K
+    q = 2 * n + n // 2 + n // 32
+    dq_b = n // 2 + n // 32 + 2 * n
+    dq_f = n // 2 + n // 32 + 4 * n
+    return q, dq_b, dq_f
+
+
+class Timer:
+    """CUDA-event timing of individual launches on the launching stream."""
+
+    def __init__(self, torch, stream):
+        self.torch = torch
+        self.stream = stream
+        self.pending = {}
+
+    def run(self, key, fn):
+        ev0 = self.torch.cuda.Event(enable_timing=True)
+        ev1 = self.torch.cuda.Event(enable_timing=True)
+        ev0.record(self.stream)
+        fn()
+        ev1.record(self.stream)
+        self.pending.setdefault(key, []).append((ev0, ev1))
+
+    def avg_ms(self, key):
+        evs = self.pending.get(key, [])
+        if not evs:
+            return None
+        return sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+
+
+def l2_flush(torch, buf):
+    buf.zero_()
+
+
+def oracle_cpu_sample(rows, seconds_target=10.0):
+    """Time the CPU oracle (single thread, as it stands) on `rows` rows of the
+    [8*2048, 7168] workload: quantize + dequantize bf16 + dequantize fp32."""
+    import numpy as np
+    import oracle
+    from fp8_microscaling_quantization_b200 import synth
+    w = synth.expert_weights(E=1, N=rows, K=K, zero_blocks=4, seed=20260002).reshape(rows, K)
+    t0 = time.perf_counter()
+    p, s = oracle.quantize_mxfp4(w)
+    oracle.dequantize_mxfp4(p, s, out_dtype=oracle.BF16)
+    oracle.dequantize_mxfp4(p, s, out_dtype=oracle.F32)
+    dt = time.perf_counter() - t0
+    n = rows * K
+    nbytes = (2 * n + n // 2 + n // 32) + (n // 2 + n // 32 + 2 * n) + (n // 2 + n // 32 + 4 * n)
+    return nbytes, dt
+
+
+def run_cpu_baseline():
+    rows = 128
+    nbytes, dt = oracle_cpu_sample(rows)
+    # scale the sample to about 10 s of CPU work
+    rows2 = int(max(128, min(8192, rows * 10.0 / max(dt, 1e-3))))
+    nbytes, dt = oracle_cpu_sample(rows2)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows2} rows x 7168 of the MXFP4 expert-weight workload (quantize + dequantize bf16 + "
+                      f"dequantize fp32), single-threaded C oracle, {dt:.1f} s"}
+
+
+# --------------------------------------------------------------- reference --
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    steps, warmup = max(1, args.steps), max(0, args.warmup)
+    rows = 64
+    for _ in range(warmup):
+        oracle_cpu_sample(rows)
+    tot_b, tot_t = 0, 0.0
+    t_start = time.perf_counter()
+    for _ in range(steps):
+        b, t = oracle_cpu_sample(rows)
+        tot_b += b
+        tot_t += t
+        if time.perf_counter() - t_start > 150:
+            break
+    val = tot_b / tot_t / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": warmup, "ms_per_step": round(tot_t / max(1, steps) * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "mxfp4_expert_weights_round_trip", "shape": [E, N, K],
+                       "sample_rows_per_step": rows},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{rows} rows x 7168 per step (quantize + dequantize bf16 + fp32)"},
+            "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- ours ---
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    from fp8_microscaling_quantization_b200 import bsq, synth
+
+    peaks, peak_kind = load_peaks()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    steps, warmup = max(1, args.steps), max(3, args.warmup)
+
+    # ---- workload: MXFP4 routed-expert weights [8, 2048, 7168] --------------
+    g = torch.Generator(device=dev)
+    g.manual_seed(20260002 + rank)
+    xs = [synth.expert_weights_torch(E, N, K, generator=g, device=dev) for _ in range(2)]
+    packed = [torch.empty((E, N, K // 2), dtype=torch.uint8, device=dev) for _ in range(3)]
+    scales = [torch.empty((E, N, K // 32), dtype=torch.uint8, device=dev) for _ in range(3)]
+    yb = torch.empty((E, N, K), dtype=torch.bfloat16, device=dev)
+    yf = torch.empty((E, N, K), dtype=torch.float32, device=dev)
+    for i in range(3):
+        bsq.bsq_quantize_mxfp4(xs[i % 2], packed=packed[i], scales=scales[i])
+    torch.cuda.synchronize()
+
+    timer = Timer(torch, stream)
+
+    def step(i, timed):
+        q = lambda: bsq.bsq_quantize_mxfp4(xs[i % 2], packed=packed[i % 3], scales=scales[i % 3])
+        d1 = lambda: bsq.bsq_dequantize_mxfp4(packed[(i + 1) % 3], scales[(i + 1) % 3], y=yb)
+        d2 = lambda: bsq.bsq_dequantize_mxfp4(packed[(i + 2) % 3], scales[(i + 2) % 3], y=yf)
+        if timed:
+            timer.run("mx_quant", q)
+            timer.run("mx_dequant_bf16", d1)
+            timer.run("mx_dequant_fp32", d2)
+        else:
+            q(), d1(), d2()
+
+    for i in range(warmup):
+        step(i, False)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_soak = time.time()
+    i = 0
+    while time.time() - t_soak < 1.0:  # keep the GPU under this load while clocks settle
+        step(i, False)
+        i += 1
+        if i % 50 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev_start = torch.cuda.Event(enable_timing=True)
+    ev_end = torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    ev_start.record(stream)
+    for i in range(steps):
+        step(i, True)
+    ev_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    clocks.stop()
+    region_ms = ev_start.elapsed_time(ev_end)
+    if world > 1:
+        t = torch.tensor([region_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        region_ms = float(t.item())
+    ms_per_step = region_ms / steps
+    qb, db, fb = mx_bytes()
+    step_bytes = qb + db + fb
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    kern = {}
+    for key, nbytes in (("mx_quant", qb), ("mx_dequant_bf16", db), ("mx_dequant_fp32", fb)):
+        ms = timer.avg_ms(key)
+        kern[key] = {"ms": round(ms, 5), "bytes": nbytes, "GB/s": round(nbytes / ms / 1e6, 1),
+                     "frac_hbm": round(nbytes / ms / 1e6 / peaks["hbm_gbs"], 4)}
+    dom = max(kern, key=lambda k: kern[k]["ms"])
+    roof = {"kernel": dom, "bound": "hbm", "achieved": kern[dom]["GB/s"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": kern[dom]["frac_hbm"], "traffic": traffic_from_profiles(dom),
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback"}
+
+    # ---- end to end through the public API with pinned host buffers ---------
+    e2e = None
+    if rank == 0 or world > 1:
+        e2e = measure_e2e(torch, bsq, xs[0], stream, steps=min(steps, 10))
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": steps,
+            "warmup": warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "mxfp4_expert_weights_round_trip: bf16 [8,2048,7168] -> int8 packed + e8m0 "
+                                   "-> bf16 and fp32", "l2": "inputs and outputs larger than L2; dequantize reads "
+                                   "packed buffers from 3 rotating slots", "parallelism": f"replicas x{world}",
+                       "frac_hbm_step": round(value / world / peaks["hbm_gbs"], 4)},
+            "roofline": roof, "kernels": kern, "gpu_launches": 3 * steps,
+            "clocks": clocks.summary(t_soak, t_wall1)}
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and rank == 0 and not args.no_cpu:
+        try:
+            line["cpu_baseline"] = run_cpu_baseline()
+        except Exception as ex:  # report, never hide
+            line["cpu_baseline"] = {"unavailable": f"{type(ex).__name__}: {ex}"}
+    if not args.no_extra and world == 1:
+        only = set(filter(None, args.only.split(",")))
+        line["extra"] = run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def measure_e2e(torch, bsq, x_dev, stream, steps):
+    """Quantize + dequantize through the C ABI with the step's input copied from
+    pinned host memory and every output copied back, inside the timed region."""
+    xh = x_dev.cpu().pin_memory()
+    xd = torch.empty_like(x_dev)
+    p = torch.empty((E, N, K // 2), dtype=torch.uint8, device=x_dev.device)
+    s = torch.empty((E, N, K // 32), dtype=torch.uint8, device=x_dev.device)
+    yb = torch.empty((E, N, K), dtype=torch.bfloat16, device=x_dev.device)
+    yf = torch.empty((E, N, K), dtype=torch.float32, device=x_dev.device)
+    ph, sh = torch.empty_like(p, device="cpu").pin_memory(), torch.empty_like(s, device="cpu").pin_memory()
+    ybh = torch.empty_like(yb, device="cpu").pin_memory()
+    yfh = torch.empty_like(yf, device="cpu").pin_memory()
+
+    def one():
+        xd.copy_(xh, non_blocking=True)
+        bsq.bsq_quantize_mxfp4(xd, packed=p, scales=s)
+        bsq.bsq_dequantize_mxfp4(p, s, y=yb)
+        bsq.bsq_dequantize_mxfp4(p, s, y=yf, out_dtype=bsq.DType.FP32)
+        ph.copy_(p, non_blocking=True)
+        sh.copy_(s, non_blocking=True)
+        ybh.copy_(yb, non_blocking=True)
+        yfh.copy_(yf, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    qb, db, fb = mx_bytes()
+    h2d = xh.numel() * 2
+    d2h = ph.numel() + sh.numel() + ybh.numel() * 2 + yfh.numel() * 4
+    return {"value": round((qb + db + fb) / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3)}
+
+
+# ------------------------------------------------------------- sub-measures -
+
+def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
+    out = {}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    hbm = peaks["hbm_gbs"]
+
+    def timed(fn, iters, cold):
+        t = Timer(torch, stream)
+        for _ in range(3):
+            fn()
+        for _ in range(iters):
+            if cold:
+                l2_flush(torch, flush)
+            t.run("k", fn)
+        torch.cuda.synchronize()
+        return t.avg_ms("k")
+
+    def rec(ms, nbytes):
+        return {"us": round(ms * 1e3, 2), "bytes": nbytes, "GB/s": round(nbytes / ms / 1e6, 1),
+                "frac_hbm": round(nbytes / ms / 1e6 / hbm, 4)}
+
+    want = (lambda s: not only or s in only)
+
+    if want("nvfp4"):
+        g = torch.Generator(device=dev)
+        g.manual_seed(20260001)
+        x = synth.nvfp4_matrix_torch(256, 2048, generator=g, device=dev)
+        p, s, r = bsq.bsq_quantize_nvfp4(x)
+        y = torch.empty_like(x)
+        n = x.numel()
+        nb = 2 * n + n // 2 + n // 16 + 4 * 256
+        out["nvfp4_256x2048"] = {
+            "quantize": rec(timed(lambda: bsq.bsq_quantize_nvfp4(x, packed=p, scales=s, row_scale_out=r), 50, True), nb),
+            "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_nvfp4(p, s, r, y=y), 50, True), nb),
+            "note": "latency-bound (1.3 MB); L2 flushed before every launch"}
+
+    if want("cache"):
+        g = torch.Generator(device=dev)
+        g.manual_seed(20260003)
+        cases = [("fp8_b32_4x8192x512", 0, 32, (4, 8192, 512)), ("mxfp4_b32_4x8192x128", 1, 32, (4, 8192, 128)),
+                 ("nvfp4_b16_4x2048x512", 2, 16, (4, 2048, 512)), ("fp8_b32_4x2048x520", 0, 32, (4, 2048, 520)),
+                 ("mxfp4_b32_4x2048x520", 1, 32, (4, 2048, 520)), ("nvfp4_b16_4x2048x520", 2, 16, (4, 2048, 520))]
+        res = {}
+        for name, fmt, blk, shp in cases:
+            x = synth.cache_acts_torch(*shp, generator=g, device=dev)
+            y = torch.empty_like(x)
+            nb = 2 * 2 * x.numel()
+            res[name] = rec(timed(lambda: bsq.bsq_quantize_cache(x, fmt, blk, y=y), 30, True), nb)
+        gsrc = torch.randn((4, 8192, 512), generator=g, device=dev).to(torch.bfloat16)
+        gdst = torch.empty_like(gsrc)
+        res["ste_backward_aliased"] = {"us": 0.0, "bytes": 0, "note": "identity: no launch"}
+        res["ste_backward_copy_4x8192x512"] = rec(
+            timed(lambda: bsq.bsq_quantize_cache_backward(gsrc, gdst), 30, True), 2 * 2 * gsrc.numel())
+        res["note"] = "L2 flushed before every launch (tensors of 8-34 MB)"
+        out["quantize_cache"] = res
+
+    if want("linear"):
+        g = torch.Generator(device=dev)
+        g.manual_seed(20260004)
+        x = synth.linear_weight_torch(7168, 18432, generator=g, device=dev)
+        up = synth.linear_weight_torch(7168, 18432, generator=g, device=dev)
+        cat = torch.cat([x, up], 0)
+        del up
+        n = x.numel()
+        p = torch.empty((7168, 18432 // 2), dtype=torch.uint8, device=dev)
+        s = torch.empty((7168, 18432 // 16), dtype=torch.uint8, device=dev)
+        r = torch.empty((7168,), dtype=torch.float32, device=dev)
+        t = torch.empty((1,), dtype=torch.float32, device=dev)
+        scratch = torch.empty((bsq.bsq_nvfp4_tensor_scratch_bytes(7168, 18432),), dtype=torch.uint8, device=dev)
+        pc = torch.empty((2 * 7168, 18432 // 2), dtype=torch.uint8, device=dev)
+        sc = torch.empty((2 * 7168, 18432 // 16), dtype=torch.uint8, device=dev)
+        rc = torch.full((2 * 7168,), 1e-5, dtype=torch.float32, device=dev)
+        rco = torch.empty_like(rc)
+        nb_row = 2 * n + n // 2 + n // 16 + 4 * 7168
+        nb_tensor = 4 * n + n // 2 + n // 16 + 4
+        nb_gu = 2 * (2 * n) + (2 * n) // 2 + (2 * n) // 16 + 2 * 4 * 14336
+        y = torch.empty((7168, 18432), dtype=torch.bfloat16, device=dev)
+        nb_dq = n // 2 + n // 16 + 4 * 7168 + 2 * n
+        out["nvfp4_linear_7168x18432"] = {
+            "modelopt_tensor_scale": rec(timed(lambda: bsq.bsq_quantize_nvfp4_tensor(
+                x, packed=p, scales=s, tensor_scale=t, scratch=scratch), 10, False), nb_tensor),
+            "per_row_scale": rec(timed(lambda: bsq.bsq_quantize_nvfp4(x, packed=p, scales=s, row_scale_out=r),
+                                       10, False), nb_row),
+            "gate_up_given_row_scales_14336x18432": rec(timed(lambda: bsq.bsq_quantize_nvfp4(
+                cat, row_scale_in=rc, packed=pc, scales=sc, row_scale_out=rco), 10, False), nb_gu),
+            "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_nvfp4(p, s, r, y=y), 10, False), nb_dq),
+            "note": "inputs larger than L2; per-tensor counts two reads of the input"}
+        del x, cat, y
+
+    if want("gemm"):
+        try:
+            out["grouped_gemm"] = bench_gemm(torch, bsq, synth, dev, stream, peaks, peak_kind)
+        except bsq.BsqError as e:
+            out["grouped_gemm"] = {"unavailable": str(e)}
+    return out
+
+
+def bench_gemm(torch, bsq, synth, dev, stream, peaks, peak_kind):
+    import numpy as np
+    T, Kd, Nd, Ed = 16384, 7168, 2048, 32
+    rng = np.random.default_rng(20260005)
+    offs_np = synth.zipf_offs(rng, T, Ed)
+    g = torch.Generator(device=dev)
+    g.manual_seed(20260005)
+    x = torch.randn((T, Kd), generator=g, device=dev).to(torch.bfloat16)
+    go = torch.randn((T, Nd), generator=g, device=dev).to(torch.bfloat16)
+    w = (torch.randn((Ed, Nd, Kd), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    mx_p, mx_s = bsq.bsq_quantize_mxfp4(w)
+    nv_p, nv_s, nv_r = bsq.bsq_quantize_nvfp4(w)
+    del w
+    offs = torch.from_numpy(offs_np).to(dev)
+    flops = 2.0 * T * Nd * Kd
+    out_f = torch.empty((T, Nd), dtype=torch.bfloat16, device=dev)
+    out_b = torch.empty((T, Kd), dtype=torch.bfloat16, device=dev)
+    err = torch.zeros((1,), dtype=torch.int32, device=dev)
+    res = {"flop_per_launch": flops, "offs": offs_np.tolist()}
+    peak = peaks["bf16_tflops"]
+    for fmt_name, fmt, p, s, r in (("mxfp4", bsq.Format.MXFP4, mx_p, mx_s, None),
+                                   ("nvfp4", bsq.Format.NVFP4, nv_p, nv_s, nv_r)):
+        for dname, d, a, o in (("fwd", bsq.Direction.FWD, x, out_f), ("bwd", bsq.Direction.BWD, go, out_b)):
+            fn = lambda: bsq.bsq_grouped_mm_fp4(fmt, d, a, p, s, r, offs, out=o, err=err)
+            t = Timer(torch, stream)
+            for _ in range(3):
+                fn()
+            for _ in range(10):
+                t.run("k", fn)
+            torch.cuda.synchronize()
+            ms = t.avg_ms("k")
+            tf = flops / (ms * 1e-3) / 1e12
+            res[f"{fmt_name}_{dname}"] = {"us": round(ms * 1e3, 1), "TFLOP/s": round(tf, 1),
+                                          "frac_bf16": round(tf / peak, 4)}
+    res["err_word"] = int(err.item())
+    res["peak"] = f"{peak} TFLOP/s bf16 dense ({peak_kind}, burst)"
+    return res
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,138 @@
+// formats.cuh -- device-side encode/decode of the microscaling element and
+// scale formats, written from the format definitions:
+//   e2m1      1 sign, 2 exponent (bias 1), 1 mantissa bit: magnitudes
+//             {0, 0.5, 1, 1.5, 2, 3, 4, 6}; the NeMo AutoModel mxfp4 page's
+//             _FP4_E2M1_TABLE decodes code 8 to +0.0.
+//   e4m3fn    1 sign, 4 exponent (bias 7), 3 mantissa bits, subnormals,
+//             max 448, S.1111.111 = NaN, no infinity.
+//   e8m0fnu   unsigned biased exponent: 2**(code - 127), 0xFF = NaN.
+// All arithmetic is IEEE binary32 round-to-nearest-even with subnormals kept
+// (the library is built without fast-math / flush-to-zero).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+namespace bsq {
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two binary32 -> packed bf16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Exponent of a binary32 as stored (biased), 0 for zero / subnormal.
+__device__ __forceinline__ int f32_biased_exp(float a) { return (__float_as_uint(a) >> 23) & 0xFF; }
+
+// floor(log2(a)) for finite a > 0, exact, subnormals included.
+__device__ __forceinline__ int floor_log2_exact(float a) {
+    uint32_t b = __float_as_uint(a) & 0x7FFFFFFFu;
+    int e = (int)(b >> 23);
+    if (e != 0) return e - 127;
+    // subnormal: value = m * 2**-149, floor(log2) = index of the top set bit - 149
+    return (31 - __clz((int)b)) - 149;
+}
+
+// 2**e as a binary32 for e in [-149, 127] (subnormal results built exactly).
+__device__ __forceinline__ float exp2_int(int e) {
+    if (e >= -126) return __uint_as_float((uint32_t)(e + 127) << 23);
+    return __uint_as_float(1u << (e + 149));
+}
+
+// Round a positive normal binary32 up to a power of two.
+__device__ __forceinline__ float pow2_ceil_normal(float a) {
+    uint32_t b = __float_as_uint(a);
+    if ((b & 0x007FFFFFu) == 0) return a;
+    return __uint_as_float((b & 0x7F800000u) + 0x00800000u);
+}
+
+// ------------------------------------------------------------------ e4m3 --
+
+// Nearest finite e4m3 code, ties to even, saturating at 448 (software; used
+// for block scales, one per block).  The quantum of a value's e4m3 binade is
+// 2**(max(floor(log2 a), -6) - 3); the code is (binade + 6) * 8 + the value in
+// quanta rounded to an integer, which carries into the exponent field by
+// itself when the rounding reaches the next binade.
+__device__ __forceinline__ uint32_t e4m3_encode_sw(float x) {
+    uint32_t sign = (__float_as_uint(x) >> 24) & 0x80u;
+    float a = fabsf(x);
+    if (!(a < 448.0f)) return sign | 0x7Eu;
+    int e = f32_biased_exp(a) - 127;
+    if (e < -6) e = -6;
+    float m = rintf(a * exp2_int(3 - e));  // exact scaling by a power of two
+    return sign | (uint32_t)((e + 6) * 8 + (int)m);
+}
+
+__device__ __forceinline__ float e4m3_decode(uint32_t c) {
+    uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    float v;
+    if (e == 0) v = (float)m * 0.001953125f;  // m * 2**-9
+    else v = __uint_as_float(((e + 120u) << 23) | (m << 20));
+    if (e == 15u && m == 7u) v = __uint_as_float(0x7FC00000u);
+    return (c & 0x80u) ? -v : v;
+}
+
+// Two binary32 -> two e4m3 bytes (hardware cvt, round to nearest even,
+// saturating to +-448): `lo` in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2_encode_hw(float lo, float hi) {
+    uint32_t out;
+    asm("{\n\t.reg .b16 t;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\t"
+        "cvt.u32.u16 %0, t;\n\t}"
+        : "=r"(out)
+        : "f"(hi), "f"(lo));
+    return out;
+}
+
+// Two e4m3 bytes (low half of w16) -> two binary32 (exact, via f16).
+__device__ __forceinline__ float2 e4m3x2_decode_hw(uint32_t w16) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 t;\n\t"
+        "cvt.u16.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(h2)
+        : "r"(w16));
+    __half2 h = *reinterpret_cast<__half2*>(&h2);
+    return __half22float2(h);
+}
+
+// ------------------------------------------------------------------ e2m1 --
+
+// Four pairs of binary32 -> four bytes of packed e2m1 (hardware cvt, round to
+// nearest even, saturating to +-6).  v[2i] goes to the low nibble of byte i.
+__device__ __forceinline__ uint32_t e2m1x8_encode_hw(const float v[8]) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return out;
+}
+
+// e2m1 code -> binary32.  Magnitude m: 0 and 1 are 0 and 0.5; m >= 2 is
+// (1 + (m & 1) / 2) * 2**((m >> 1) - 1).  Code 8 decodes to +0.0.
+__device__ __forceinline__ float e2m1_decode(uint32_t c) {
+    uint32_t m = c & 7u;
+    uint32_t bits = (m >= 2u) ? ((((m >> 1) + 126u) << 23) | ((m & 1u) << 22))
+                              : (m == 1u ? 0x3F000000u : 0u);
+    if ((c & 8u) && m) bits |= 0x80000000u;
+    return __uint_as_float(bits);
+}
+
+// e8m0 byte -> 2**(code - 127) as binary32 (code 0 is the subnormal 2**-127,
+// 0xFF is NaN).
+__device__ __forceinline__ float e8m0_decode(uint32_t c) {
+    c &= 0xFFu;
+    if (c == 0xFFu) return __uint_as_float(0x7FC00000u);
+    if (c == 0u) return __uint_as_float(0x00400000u);
+    return __uint_as_float(c << 23);
+}
+
+}  // namespace bsq

@@ -119,3 +119,51 @@ def moe_problem(T=16384, K=7168, N=2048, E=32, seed=None, with_weights=True):
         del wf
     go = to_bf16_bits(rng.standard_normal((T, N), dtype=np.float32))
     return {"x": x, "offs": offs, "w": w, "grad_out": go}
+
+
+# --------------------------------------------------------------------------
+# Device-side variants for the benchmark: the same recipes drawn with torch's
+# CUDA generator (same distributions and structure; different random numbers
+# from the numpy variants above, which feed the parity tests).
+
+def _bf16(t):
+    return t.to(torch.bfloat16)
+
+
+def nvfp4_matrix_torch(rows=256, cols=2048, generator=None, device="cuda"):
+    x = torch.randn((rows, cols), generator=generator, device=device)
+    n = int(round(0.01 * x.numel()))
+    idx = torch.randperm(x.numel(), generator=generator, device=device)[:n]
+    x.view(-1)[idx] *= 20.0
+    return _bf16(x)
+
+
+def expert_weights_torch(E=8, N=2048, K=7168, zero_blocks=16, generator=None, device="cuda", block=32):
+    w = torch.randn((E, N, K), generator=generator, device=device)
+    w *= 0.02
+    lo, hi = float(np.log(0.5)), float(np.log(2.0))
+    f = torch.empty((E, N, 1), device=device).uniform_(lo, hi, generator=generator).exp_()
+    w *= f
+    nb = N * (K // block)
+    for e in range(E):
+        pick = torch.randperm(nb, generator=generator, device=device)[:zero_blocks].tolist()
+        for p in pick:
+            r, b = divmod(int(p), K // block)
+            w[e, r, b * block:(b + 1) * block] = 0.0
+    return _bf16(w)
+
+
+def cache_acts_torch(B=4, T=8192, C=512, generator=None, device="cuda"):
+    x = torch.randn((B, T, C), generator=generator, device=device)
+    f = torch.empty((1, 1, C), device=device).uniform_(float(np.log(0.1)), float(np.log(10.0)),
+                                                       generator=generator).exp_()
+    return _bf16(x * f)
+
+
+def linear_weight_torch(out=7168, inp=18432, generator=None, device="cuda"):
+    w = torch.randn((out, inp), generator=generator, device=device)
+    w *= 0.01
+    n = int(round(0.001 * w.numel()))
+    idx = torch.randint(0, w.numel(), (n,), generator=generator, device=device)
+    w.view(-1)[idx] *= 50.0
+    return _bf16(w)

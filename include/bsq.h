@@ -1,0 +1,175 @@
+/*
+ * bsq.h -- C ABI of libbsq: block-scaled microscaling quantization for
+ * NVIDIA B200 (sm_100a).
+ *
+ * Formats (NeMo AutoModel API pages "nemo_automodel.components.quantization.nvfp4",
+ * "...quantization.mxfp4" and "...models.deepseek_v41.quantization"):
+ *   NVFP4 -- e2m1 codes, one float8_e4m3fn scale per 16 columns and one fp32
+ *            scale per row (or per tensor, the ModelOpt checkpoint layout).
+ *   MXFP4 -- e2m1 codes, one float8_e8m0fnu scale per 32 columns.
+ *   FP8   -- float8_e4m3fn codes with a power-of-two block scale, stored as an
+ *            e8m0 exponent byte per block.
+ * Two e2m1 codes share a byte: the even column in the low nibble, the odd
+ * column in the high nibble.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are contiguous and row-major; "rows" is the product of all
+ *     leading dimensions and K (or C) the last dimension.
+ *   - Every data pointer is a DEVICE pointer, owned by the caller.  The
+ *     library never allocates or frees device memory and keeps no state
+ *     between calls; outputs are written in place, so buffer addresses stay
+ *     stable (CUDA graph friendly).  Inputs are never modified.
+ *   - Work is enqueued on `stream` and is asynchronous.  Only argument
+ *     validation runs on the host; a rejected call launches nothing.
+ *   - Return value: BSQ_OK, or an error code; bsq_last_error() returns a
+ *     thread-local description of the last failure.
+ *   - bf16 tensors are passed as their 16-bit patterns.
+ *   - NaN or infinite inputs are outside the contract: the kernels finish and
+ *     the outputs are unspecified.
+ */
+#ifndef BSQ_H
+#define BSQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t; NULL is the legacy default stream. */
+typedef void* bsq_stream_t;
+
+typedef enum {
+    BSQ_OK = 0,
+    BSQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, K not a whole number of blocks, ... */
+    BSQ_ERR_UNSUPPORTED = 2, /* dtype / format / block combination not implemented */
+    BSQ_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed (see bsq_last_error) */
+    BSQ_ERR_DEVICE = 4       /* a kernel reported bad data through its device error word */
+} bsq_status;
+
+typedef enum { BSQ_BF16 = 0, BSQ_FP32 = 1 } bsq_dtype;
+typedef enum { BSQ_FP8 = 0, BSQ_MXFP4 = 1, BSQ_NVFP4 = 2 } bsq_format;
+typedef enum { BSQ_FWD = 0, BSQ_BWD = 1 } bsq_dir;
+
+/* Bits of the device error word written by bsq_grouped_mm_fp4. */
+#define BSQ_DEVERR_BAD_OFFS 1u  /* offs not non-decreasing, negative, or offs[E-1] > T */
+#define BSQ_DEVERR_TIMEOUT 2u   /* a pipeline wait gave up after its time limit (about 1 s) */
+
+const char* bsq_status_string(bsq_status s);
+const char* bsq_last_error(void);
+int bsq_version(void);
+
+/* ---------------------------------------------------------------- NVFP4 --
+ * nvfp4 page, quantize_nvfp4: along the last dim (K % 16 == 0, else
+ * BSQ_ERR_INVALID_ARG -- the page's _check_last_dim), ModelOpt convention
+ *   global      = amax(row) / (6 * 448)            (row_scale_in == NULL)
+ *   block_scale = e4m3(amax(block) / 6 / global)    floored at 2**-9 before the cast
+ *   code        = round_to_e2m1(w / (block_scale * global))
+ * e4m3 and e2m1 rounding is to nearest, ties to even, saturating.  An all-zero
+ * row (or a given row scale of 0) yields scale bytes 0x00 and codes 0.
+ *   x             [rows, K] bf16 or fp32 (xt)
+ *   row_scale_in  [rows] fp32 row scales to use instead of the amax rule, or NULL
+ *   packed        [rows, K/2] uint8 out
+ *   scales_e4m3   [rows, K/16] float8_e4m3fn out
+ *   row_scale_out [rows] fp32 out (the row scale used; may equal row_scale_in) */
+bsq_status bsq_quantize_nvfp4(const void* x, bsq_dtype xt, int64_t rows, int64_t K,
+                              const float* row_scale_in, uint8_t* packed, uint8_t* scales_e4m3,
+                              float* row_scale_out, bsq_stream_t stream);
+
+/* nvfp4 page, quantize_nvfp4_modelopt: one tensor scale amax(x) / (6 * 448)
+ * for the whole [rows, K] matrix (the checkpoint's weight_scale_2), then the
+ * per-row algorithm above with that scale on every row.  Two passes over x.
+ *   tensor_scale_out  device fp32 scalar out
+ *   scratch           caller-owned device buffer of at least
+ *                     bsq_nvfp4_tensor_scratch_bytes(rows, K) bytes, 16-byte
+ *                     aligned; it holds per-block partial maxima between the
+ *                     two passes and needs no initialisation. */
+size_t bsq_nvfp4_tensor_scratch_bytes(int64_t rows, int64_t K);
+bsq_status bsq_quantize_nvfp4_tensor(const void* x, bsq_dtype xt, int64_t rows, int64_t K,
+                                     uint8_t* packed, uint8_t* scales_e4m3, float* tensor_scale_out,
+                                     void* scratch, size_t scratch_bytes, bsq_stream_t stream);
+
+/* nvfp4 page, dequantize_nvfp4: y = e2m1 * float(e4m3) * row_scale with
+ * binary32 intermediates left to right and one final rounding to yt.
+ *   packed [rows, K/2], scales_e4m3 [rows, K/16], row_scale [rows] fp32,
+ *   y [rows, K] bf16 or fp32 (yt). */
+bsq_status bsq_dequantize_nvfp4(const uint8_t* packed, const uint8_t* scales_e4m3,
+                                const float* row_scale, int64_t rows, int64_t K, void* y,
+                                bsq_dtype yt, bsq_stream_t stream);
+
+/* ---------------------------------------------------------------- MXFP4 --
+ * mxfp4 page, quantize_mxfp4: K % 32 == 0; per 32-block scale
+ * 2**(floor(log2(amax)) - 2) (exact floor; an all-zero block takes 2**-127;
+ * exponent clamped to [-127, 127]), stored as the e8m0 byte exponent + 127;
+ * code = round_to_e2m1(w / scale).
+ *   x [rows, K] bf16 or fp32; packed [rows, K/2] (int8 container, same bits);
+ *   scales_e8m0 [rows, K/32]. */
+bsq_status bsq_quantize_mxfp4(const void* x, bsq_dtype xt, int64_t rows, int64_t K,
+                              uint8_t* packed, uint8_t* scales_e8m0, bsq_stream_t stream);
+
+/* mxfp4 page, dequantize_mxfp4: y = e2m1 * 2**(scale byte - 127) (exact;
+ * scale byte 0xFF is NaN). */
+bsq_status bsq_dequantize_mxfp4(const uint8_t* packed, const uint8_t* scales_e8m0, int64_t rows,
+                                int64_t K, void* y, bsq_dtype yt, bsq_stream_t stream);
+
+/* ------------------------------------------------------------------ FP8 --
+ * Stored form of the cache page's "fp8" representation: block of `block`
+ * (16 or 32) columns, scale p = pow2ceil(max(amax / 448, 2**-126))
+ * (deepseek_v41 quantization page, _power_of_two_ceiling), e4m3 code =
+ * round(x / p) to nearest even; the scale is stored as log2(p) + 127.
+ *   codes_e4m3 [rows, K] uint8 out; scales_e8m0 [rows, K/block] out. */
+bsq_status bsq_quantize_fp8(const void* x, bsq_dtype xt, int64_t rows, int64_t K, int block,
+                            uint8_t* codes_e4m3, uint8_t* scales_e8m0, bsq_stream_t stream);
+
+/* y = float(e4m3) * 2**(scale byte - 127), one rounding to yt. */
+bsq_status bsq_dequantize_fp8(const uint8_t* codes_e4m3, const uint8_t* scales_e8m0, int64_t rows,
+                              int64_t K, int block, void* y, bsq_dtype yt, bsq_stream_t stream);
+
+/* ------------------------------------------------------- quantize_cache --
+ * deepseek_v41 quantization page, quantize_cache / _CacheQuantization.forward:
+ * quantize then dequantize every group of `block` consecutive channels of the
+ * [rows, C] input, returning a new tensor of the input dtype.  Any C >= 0: a
+ * final partial group is zero-padded internally.  Scale rules:
+ *   BSQ_FP8   -- p = pow2ceil(max(amax/448, 2**-126)), e4m3 values
+ *   BSQ_MXFP4 -- p = pow2ceil(max(amax/6,   2**-126)), e2m1 values
+ *   BSQ_NVFP4 -- the per-row NVFP4 rule above over the zero-padded row
+ * block is 16 or 32.  x and y must not overlap (the input is never modified). */
+bsq_status bsq_quantize_cache(bsq_format fmt, int block, const void* x, void* y, bsq_dtype t,
+                              int64_t rows, int64_t C, bsq_stream_t stream);
+
+/* _CacheQuantization.backward: the straight-through gradient is the identity.
+ * grad_in == grad_out is a no-op; otherwise one device-to-device copy of
+ * n_elems elements of dtype t. */
+bsq_status bsq_quantize_cache_backward(const void* grad_out, void* grad_in, bsq_dtype t,
+                                       int64_t n_elems, bsq_stream_t stream);
+
+/* ------------------------------------------------------- grouped GEMM ----
+ * nvfp4 page NVFP4GroupedMM / mxfp4 page MXFP4GroupedMM, with the weights
+ * dequantized on the fly inside the kernel (never materialised in HBM):
+ *   expert e owns rows [offs[e-1], offs[e]) of the activations (offs[-1] = 0);
+ *   BSQ_FWD: out[t, :]    = x[t, :]        @ W_e^T   a = x [T, K],        out [T, N]
+ *   BSQ_BWD: grad_x[t, :] = grad_out[t, :] @ W_e     a = grad_out [T, N], out [T, K]
+ * with W_e the dequantized [N, K] weight.  No weight gradient (frozen base).
+ *   fmt         BSQ_MXFP4 (scales e8m0 [E, N, K/32], row_scale NULL) or
+ *               BSQ_NVFP4 (scales e4m3 [E, N, K/16], row_scale fp32 [E, N])
+ *   a, out      bf16; fp32 accumulation on the tensor cores
+ *   packed      uint8 [E, N, K/2]
+ *   offs        int32 [E] cumulative token counts, on the device
+ *   err         device uint32 word; the caller zeroes it before the call and
+ *               reads it after synchronising: BSQ_DEVERR_* bits.  With a bad
+ *               offs the output is undefined.
+ * Rows at or past offs[E-1] are written as zero.  Requirements:
+ * N % 256 == 0 for BSQ_FWD and K % 256 == 0 for BSQ_BWD (the output tile
+ * width); K % 64 == 0 and N % 64 == 0 (contraction tiles); x, packed and out
+ * 16-byte aligned.  Other shapes return BSQ_ERR_UNSUPPORTED. */
+bsq_status bsq_grouped_mm_fp4(bsq_format fmt, bsq_dir dir, const void* a, const uint8_t* packed,
+                              const uint8_t* scales, const float* row_scale, const int32_t* offs,
+                              int E, int64_t T, int64_t N, int64_t K, void* out, uint32_t* err,
+                              bsq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSQ_H */

@@ -1,0 +1,115 @@
+"""C-ABI boundary tests that need no GPU: the library loads, exports every
+entry point include/bsq.h declares, and rejects bad arguments on the host
+before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "bsq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp8_microscaling_quantization_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_hot_path():
+    names = declared_entry_points()
+    for n in ["bsq_quantize_nvfp4", "bsq_quantize_nvfp4_tensor", "bsq_dequantize_nvfp4", "bsq_quantize_mxfp4",
+              "bsq_dequantize_mxfp4", "bsq_quantize_fp8", "bsq_dequantize_fp8", "bsq_quantize_cache",
+              "bsq_quantize_cache_backward", "bsq_grouped_mm_fp4"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_entry_points() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_entry_point():
+    from fp8_microscaling_quantization_b200 import bsq
+    assert set(declared_entry_points()) <= set(bsq.EXPORTED)
+    for n in declared_entry_points():
+        assert callable(getattr(bsq, n))
+
+
+def test_status_strings(lib):
+    lib.bsq_status_string.restype = ctypes.c_char_p
+    assert lib.bsq_status_string(0) == b"ok"
+    assert lib.bsq_status_string(1) == b"invalid argument"
+    assert lib.bsq_version() >= 1
+
+
+# --- host-side validation (nothing is launched for a rejected call) --------
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below is rejected first
+I64 = ctypes.c_int64
+INVALID, UNSUPPORTED = 1, 2
+
+
+def _err(lib):
+    lib.bsq_last_error.restype = ctypes.c_char_p
+    return lib.bsq_last_error().decode()
+
+
+def test_nvfp4_rejects_ragged_k(lib):
+    rc = lib.bsq_quantize_nvfp4(FAKE, 0, I64(4), I64(24), None, FAKE, FAKE, FAKE, None)
+    assert rc == INVALID and "16-column blocks" in _err(lib)
+
+
+def test_mxfp4_rejects_ragged_k(lib):
+    assert lib.bsq_quantize_mxfp4(FAKE, 0, I64(4), I64(48), FAKE, FAKE, None) == INVALID
+    assert lib.bsq_dequantize_mxfp4(FAKE, FAKE, I64(4), I64(48), FAKE, 0, None) == INVALID
+
+
+def test_rejects_null_and_negative(lib):
+    assert lib.bsq_quantize_nvfp4(None, 0, I64(4), I64(32), None, FAKE, FAKE, FAKE, None) == INVALID
+    assert lib.bsq_quantize_nvfp4(FAKE, 0, I64(4), I64(32), None, None, FAKE, FAKE, None) == INVALID
+    assert lib.bsq_quantize_mxfp4(FAKE, 0, I64(-1), I64(32), FAKE, FAKE, None) == INVALID
+    assert lib.bsq_dequantize_nvfp4(FAKE, None, FAKE, I64(4), I64(32), FAKE, 0, None) == INVALID
+
+
+def test_rejects_bad_dtype_format_block(lib):
+    assert lib.bsq_quantize_mxfp4(FAKE, 7, I64(4), I64(32), FAKE, FAKE, None) == UNSUPPORTED
+    assert lib.bsq_quantize_fp8(FAKE, 0, I64(4), I64(64), 8, FAKE, FAKE, None) == INVALID
+    assert lib.bsq_quantize_cache(9, 16, FAKE, ctypes.c_void_p(0x90000), 0, I64(4), I64(64), None) == UNSUPPORTED
+    assert lib.bsq_quantize_cache(0, 24, FAKE, ctypes.c_void_p(0x90000), 0, I64(4), I64(64), None) == INVALID
+
+
+def test_cache_rejects_overlap(lib):
+    rc = lib.bsq_quantize_cache(0, 32, FAKE, ctypes.c_void_p(0x10000 + 64), 0, I64(4), I64(64), None)
+    assert rc == INVALID and "overlap" in _err(lib)
+
+
+def test_misaligned_pointers_rejected(lib):
+    rc = lib.bsq_quantize_mxfp4(ctypes.c_void_p(0x10002), 0, I64(4), I64(32), FAKE, FAKE, None)
+    assert rc == INVALID and "misaligned" in _err(lib)
+
+
+def test_empty_tensors_are_no_ops(lib):
+    # zero rows: nothing to do, nothing launched, OK even with null pointers
+    assert lib.bsq_quantize_mxfp4(None, 0, I64(0), I64(32), None, None, None) == 0
+    assert lib.bsq_dequantize_fp8(None, None, I64(0), I64(64), 32, None, 0, None) == 0
+    assert lib.bsq_quantize_cache(1, 32, None, None, 0, I64(0), I64(520), None) == 0
+    assert lib.bsq_quantize_cache_backward(FAKE, FAKE, 0, I64(100), None) == 0  # aliased: identity, no copy
+
+
+def test_tensor_scratch_size(lib):
+    lib.bsq_nvfp4_tensor_scratch_bytes.restype = ctypes.c_size_t
+    n = lib.bsq_nvfp4_tensor_scratch_bytes(I64(7168), I64(18432))
+    assert n >= 4 and n % 16 == 0
+    rc = lib.bsq_quantize_nvfp4_tensor(FAKE, 0, I64(7168), I64(18432), FAKE, FAKE, FAKE, FAKE,
+                                       ctypes.c_size_t(0), None)
+    assert rc == INVALID and "scratch" in _err(lib)
