@@ -61,6 +61,7 @@ _SIGS = {
     "bsq_quantize_nvfp4": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _P, _P]),
     "bsq_nvfp4_tensor_scratch_bytes": (_SZ, [_I64, _I64]),
     "bsq_quantize_nvfp4_tensor": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
+    "bsq_quantize_nvfp4_tensor_noalloc": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _P]),
     "bsq_dequantize_nvfp4": (_I32, [_P, _P, _P, _I64, _I64, _P, _I32, _P]),
     "bsq_quantize_mxfp4": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P]),
     "bsq_dequantize_mxfp4": (_I32, [_P, _P, _I64, _I64, _P, _I32, _P]),
@@ -170,6 +171,19 @@ def bsq_quantize_nvfp4_tensor(x, packed=None, scales=None, tensor_scale=None, sc
         scratch = _empty((nbytes,), torch.uint8, x)
     _call("bsq_quantize_nvfp4_tensor", _ptr(x), _dtype_of(x), rows, K, _ptr(packed), _ptr(scales),
           _ptr(tensor_scale), _ptr(scratch), scratch.numel() * scratch.element_size(), _stream(stream))
+    return packed, scales, tensor_scale
+
+
+def bsq_quantize_nvfp4_tensor_noalloc(x, packed=None, scales=None, tensor_scale=None, stream=None):
+    """bsq_quantize_nvfp4_tensor without a scratch buffer (the library's own
+    device array holds the partial maxima; see include/bsq.h for the limits)."""
+    rows, K = _rows_k(x)
+    lead = tuple(x.shape[:-1])
+    packed = _empty(lead + (K // 2,), torch.uint8, x) if packed is None else packed
+    scales = _empty(lead + (K // 16,), torch.uint8, x) if scales is None else scales
+    tensor_scale = _empty((1,), torch.float32, x) if tensor_scale is None else tensor_scale
+    _call("bsq_quantize_nvfp4_tensor_noalloc", _ptr(x), _dtype_of(x), rows, K, _ptr(packed), _ptr(scales),
+          _ptr(tensor_scale), _stream(stream))
     return packed, scales, tensor_scale
 
 

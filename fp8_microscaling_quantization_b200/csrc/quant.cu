@@ -759,6 +759,84 @@ BSQ_API bsq_status bsq_quantize_nvfp4_tensor(const void* x, bsq_dtype xt, int64_
     return check_launch("bsq_quantize_nvfp4_tensor");
 }
 
+// ----------------------------------------------- no-allocation variant ----
+// Some callers cannot hand the library a scratch buffer: a serving engine that
+// reserves all device memory up front and forbids allocations afterwards, or a
+// plain C caller with no device allocator of its own.  For them the per-tensor
+// NVFP4 quantization can keep its per-CTA partial maxima in this file-scope
+// device array instead.  Every GPU that loads the library holds these 16 KiB
+// until the process exits.  The partial maxima are fully written by the first
+// pass before the second pass reads them, so nothing needs clearing between
+// calls.
+constexpr int kNoAllocMaxPartials = 4096;
+static __device__ __align__(256) float g_noalloc_partials[kNoAllocMaxPartials];
+
+// Device address of g_noalloc_partials, looked up once per device with that
+// device current (in host code the array's name is only a host-side handle).
+static float* noalloc_partials_ptr(bsq_status* st) {
+    static std::mutex mu;
+    static float* ptrs[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        *st = fail(BSQ_ERR_CUDA, "bsq_quantize_nvfp4_tensor_noalloc: no current device (%s)",
+                   cudaGetErrorString(e));
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (ptrs[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+        if (e != cudaSuccess || p == nullptr) {
+            *st = fail(BSQ_ERR_CUDA, "bsq_quantize_nvfp4_tensor_noalloc: cudaGetSymbolAddress failed (%s)",
+                       cudaGetErrorString(e));
+            return nullptr;
+        }
+        ptrs[dev] = (float*)p;
+    }
+    *st = BSQ_OK;
+    return ptrs[dev];
+}
+
+BSQ_API bsq_status bsq_quantize_nvfp4_tensor_noalloc(const void* x, bsq_dtype xt, int64_t rows, int64_t K,
+                                                     uint8_t* packed, uint8_t* scales_e4m3, float* tensor_scale_out,
+                                                     bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(xt));
+    BSQ_TRY(check_matrix("bsq_quantize_nvfp4_tensor_noalloc", x, rows, K, 16));
+    if (!tensor_scale_out) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor_noalloc: null tensor scale");
+    cudaStream_t st = (cudaStream_t)stream;
+    if (rows * K == 0) {
+        if (cudaMemsetAsync(tensor_scale_out, 0, sizeof(float), st) != cudaSuccess)
+            return check_launch("bsq_quantize_nvfp4_tensor_noalloc");
+        return BSQ_OK;
+    }
+    if (!packed || !scales_e4m3) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor_noalloc: null pointer");
+    if (!aligned(x, 16) || !aligned(packed, 4))
+        return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor_noalloc: misaligned pointer");
+    const int P = tensor_partials(rows, K);
+    if (P > kNoAllocMaxPartials)
+        return fail(BSQ_ERR_UNSUPPORTED,
+                    "bsq_quantize_nvfp4_tensor_noalloc: needs %d partial maxima, the built-in scratch holds %d",
+                    P, kNoAllocMaxPartials);
+    bsq_status status;
+    float* partial = noalloc_partials_ptr(&status);
+    if (!partial) return status;
+    const int64_t nchunks = rows * (K / 8);
+    const FastDiv cpr = make_fastdiv((uint32_t)(K / 8));
+    if (xt == BSQ_BF16) {
+        amax_partial_kernel<uint16_t, 4><<<P, kThreads, 0, st>>>((const uint16_t*)x, nchunks, partial);
+        BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
+        nv_flat_quant_kernel<uint16_t, 1, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(
+            (const uint16_t*)x, nchunks, cpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+    } else {
+        amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
+        BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
+        nv_flat_quant_kernel<float, 1, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(
+            (const float*)x, nchunks, cpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+    }
+    return check_launch("bsq_quantize_nvfp4_tensor_noalloc");
+}
+
 BSQ_API bsq_status bsq_dequantize_nvfp4(const uint8_t* packed, const uint8_t* scales_e4m3, const float* row_scale,
                                         int64_t rows, int64_t K, void* y, bsq_dtype yt, bsq_stream_t stream) {
     BSQ_TRY(check_dtype(yt));

@@ -90,6 +90,26 @@ bsq_status bsq_quantize_nvfp4_tensor(const void* x, bsq_dtype xt, int64_t rows, 
                                      uint8_t* packed, uint8_t* scales_e4m3, float* tensor_scale_out,
                                      void* scratch, size_t scratch_bytes, bsq_stream_t stream);
 
+/* Same computation and outputs as bsq_quantize_nvfp4_tensor, for callers
+ * that cannot provide a scratch buffer -- e.g. a serving engine that reserves
+ * all device memory at start-up and allows no allocation afterwards, or a
+ * plain C caller without a device allocator.  (The quantization pages have no
+ * counterpart: this is a property of the library, not of the method.)
+ *   - Allocates nothing: the partial maxima live in a 16 KiB array inside the
+ *     library (4096 floats), held on every GPU that loads it until exit.
+ *   - Shapes whose first pass would need more than 4096 partial maxima
+ *     (only possible on a GPU with more than 512 SMs) are rejected with
+ *     BSQ_ERR_UNSUPPORTED.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array: calls whose kernels overlap on the GPU
+ *     (concurrent streams) race and give wrong results.  Serialise them.
+ *     Nothing needs clearing between calls. */
+bsq_status bsq_quantize_nvfp4_tensor_noalloc(const void* x, bsq_dtype xt, int64_t rows, int64_t K,
+                                             uint8_t* packed, uint8_t* scales_e4m3, float* tensor_scale_out,
+                                             bsq_stream_t stream);
+
 /* nvfp4 page, dequantize_nvfp4: y = e2m1 * float(e4m3) * row_scale with
  * binary32 intermediates left to right and one final rounding to yt.
  *   packed [rows, K/2], scales_e4m3 [rows, K/16], row_scale [rows] fp32,
