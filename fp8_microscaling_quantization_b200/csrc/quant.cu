@@ -220,86 +220,6 @@ __device__ __forceinline__ void build_e2m1_lut(float2* lut) {
     __syncthreads();
 }
 
-// MXFP4 dequantize: item = 16 packed bytes = one 32-block.
-template <typename T, int U>
-__global__ void __launch_bounds__(kThreads) mx_dequant_kernel(const uint8_t* __restrict__ packed,
-                                                              const uint8_t* __restrict__ scales,
-                                                              int64_t nblocks, T* __restrict__ y) {
-    __shared__ float2 lut[256];
-    build_e2m1_lut(lut);
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nblocks; base += U * stride) {
-        uint4 w[U];
-        uint32_t sc[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t b = base + u * stride;
-            if (b < nblocks) {
-                w[u] = __ldcs(reinterpret_cast<const uint4*>(packed) + b);
-                sc[u] = scales[b];
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t b = base + u * stride;
-            if (b >= nblocks) continue;
-            const float S = e8m0_decode(sc[u]);
-            const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float v[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 t = lut[(words[q] >> (8 * i)) & 0xFFu];
-                    v[2 * i] = t.x * S;
-                    v[2 * i + 1] = t.y * S;
-                }
-                store8(y + b * 32 + q * 8, v);
-            }
-        }
-    }
-}
-
-// FP8 dequantize: item = 16 codes.
-template <typename T, int BLOCK, int U>
-__global__ void __launch_bounds__(kThreads) fp8_dequant_kernel(const uint8_t* __restrict__ codes,
-                                                               const uint8_t* __restrict__ scales,
-                                                               int64_t nitems, T* __restrict__ y) {
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nitems; base += U * stride) {
-        uint4 w[U];
-        uint32_t sc[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t it = base + u * stride;
-            if (it < nitems) {
-                w[u] = __ldcs(reinterpret_cast<const uint4*>(codes) + it);
-                sc[u] = scales[(it * 16) / BLOCK];
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t it = base + u * stride;
-            if (it >= nitems) continue;
-            const float p = e8m0_decode(sc[u]);
-            const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float v[8];
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const uint32_t word = words[2 * h + i];
-                    const float2 a = e4m3x2_decode_hw(word & 0xFFFFu);
-                    const float2 b = e4m3x2_decode_hw(word >> 16);
-                    v[4 * i + 0] = a.x * p; v[4 * i + 1] = a.y * p;
-                    v[4 * i + 2] = b.x * p; v[4 * i + 3] = b.y * p;
-                }
-                store8(y + it * 16 + h * 8, v);
-            }
-        }
-    }
-}
-
 // ----------------------------------------------------------------- NVFP4 ----
 
 // Quantize one 8-element chunk whose block partner is lane ^ 1, given the
@@ -484,44 +404,81 @@ __global__ void __launch_bounds__(kThreads) nv_flat_quant_kernel(const T* __rest
     }
 }
 
-// NVFP4 dequantize: item = 8 packed bytes = one 16-block.
-template <typename T, int U>
-__global__ void __launch_bounds__(kThreads) nv_dequant_kernel(const uint8_t* __restrict__ packed,
-                                                              const uint8_t* __restrict__ scales,
-                                                              const float* __restrict__ g, int64_t nblocks,
-                                                              FastDiv bpr, T* __restrict__ y) {
+// Dequantize (all formats).  Item = the EPI consecutive output elements of
+// one lane: 8 for bf16 output (one 16-byte store) and 4 for fp32 output (one
+// 16-byte store), so consecutive lanes write consecutive 16-byte pieces and a
+// warp store instruction covers one contiguous 512-byte span.  FP4 codes are
+// decoded through a 256-entry byte -> (low value, high value) table in shared
+// memory; e4m3 codes through the hardware cvt (exact).
+//   FMT_MX : y = e2m1 * 2**(scale - 127)
+//   FMT_NV : y = (e2m1 * e4m3(scale)) * g[row], row = block / bpr
+//   FMT_FP8: y = e4m3 * 2**(scale - 127)
+enum { FMT_FP8 = 0, FMT_MX = 1, FMT_NV = 2 };
+
+template <int FMT, typename TOUT, int BLOCK, int U>
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __restrict__ codes,
+                                                           const uint8_t* __restrict__ scales,
+                                                           const float* __restrict__ g, FastDiv bpr,
+                                                           int64_t nitems, TOUT* __restrict__ y) {
+    constexpr int EPI = (sizeof(TOUT) == 2) ? 8 : 4;         // elements per item
+    constexpr int CB = (FMT == FMT_FP8) ? EPI : EPI / 2;     // code bytes per item
     __shared__ float2 lut[256];
-    build_e2m1_lut(lut);
+    if (FMT != FMT_FP8) build_e2m1_lut(lut);
     const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nblocks; base += U * stride) {
-        uint2 w[U];
-        uint32_t sc[U];
+    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nitems; base += U * stride) {
+        uint32_t w0[U], w1[U], sc[U];
         float gr[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t b = base + u * stride;
-            if (b < nblocks) {
-                w[u] = __ldcs(reinterpret_cast<const uint2*>(packed) + b);
-                sc[u] = scales[b];
-                gr[u] = g[fdiv((uint32_t)b, bpr)];
+            const int64_t it = base + u * stride;
+            w0[u] = w1[u] = sc[u] = 0u;
+            gr[u] = 0.0f;
+            if (it < nitems) {
+                if (CB == 2) w0[u] = __ldcs(reinterpret_cast<const unsigned short*>(codes) + it);
+                else if (CB == 4) w0[u] = __ldcs(reinterpret_cast<const unsigned int*>(codes) + it);
+                else {
+                    const uint2 t = __ldcs(reinterpret_cast<const uint2*>(codes) + it);
+                    w0[u] = t.x;
+                    w1[u] = t.y;
+                }
+                const int64_t blk = (it * EPI) / BLOCK;
+                sc[u] = scales[blk];
+                if (FMT == FMT_NV) gr[u] = g[fdiv((uint32_t)blk, bpr)];
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t b = base + u * stride;
-            if (b >= nblocks) continue;
-            const float s = e4m3_decode(sc[u]);
-            const uint32_t words[2] = {w[u].x, w[u].y};
+            const int64_t it = base + u * stride;
+            if (it >= nitems) continue;
+            float v[8];
+            if (FMT == FMT_FP8) {
+                const float p = e8m0_decode(sc[u]);
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                float v[8];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 t = lut[(words[q] >> (8 * i)) & 0xFFu];
-                    v[2 * i] = __fmul_rn(__fmul_rn(t.x, s), gr[u]);
-                    v[2 * i + 1] = __fmul_rn(__fmul_rn(t.y, s), gr[u]);
+                for (int i = 0; i < EPI / 2; ++i) {
+                    const uint32_t word = (i < 2) ? w0[u] : w1[u];
+                    const float2 d = e4m3x2_decode_hw((word >> (16 * (i & 1))) & 0xFFFFu);
+                    v[2 * i] = d.x * p;
+                    v[2 * i + 1] = d.y * p;
                 }
-                store8(y + b * 16 + q * 8, v);
+            } else {
+                const float s = (FMT == FMT_MX) ? e8m0_decode(sc[u]) : e4m3_decode(sc[u]);
+#pragma unroll
+                for (int i = 0; i < EPI / 2; ++i) {
+                    const float2 t = lut[(w0[u] >> (8 * i)) & 0xFFu];
+                    if (FMT == FMT_MX) {
+                        v[2 * i] = t.x * s;
+                        v[2 * i + 1] = t.y * s;
+                    } else {
+                        v[2 * i] = __fmul_rn(__fmul_rn(t.x, s), gr[u]);
+                        v[2 * i + 1] = __fmul_rn(__fmul_rn(t.y, s), gr[u]);
+                    }
+                }
+            }
+            TOUT* dst = y + it * EPI;
+            if (sizeof(TOUT) == 2) {
+                store8(reinterpret_cast<uint16_t*>(dst), v);
+            } else {
+                __stcs(reinterpret_cast<float4*>(dst), make_float4(v[0], v[1], v[2], v[3]));
             }
         }
     }
@@ -843,16 +800,18 @@ BSQ_API bsq_status bsq_dequantize_nvfp4(const uint8_t* packed, const uint8_t* sc
     BSQ_TRY(check_matrix("bsq_dequantize_nvfp4", packed, rows, K, 16));
     if (rows * K == 0) return BSQ_OK;
     if (!scales_e4m3 || !row_scale || !y) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_nvfp4: null pointer");
-    if (!aligned(packed, 8) || !aligned(y, 16)) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_nvfp4: misaligned pointer");
-    const int64_t nblocks = rows * (K / 16);
+    if (!aligned(packed, 4) || !aligned(y, 16)) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_nvfp4: misaligned pointer");
     const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
     cudaStream_t st = (cudaStream_t)stream;
-    if (yt == BSQ_BF16)
-        nv_dequant_kernel<uint16_t, 4><<<grid_for(nblocks, 4), kThreads, 0, st>>>(packed, scales_e4m3, row_scale, nblocks,
-                                                                                 bpr, (uint16_t*)y);
-    else
-        nv_dequant_kernel<float, 4><<<grid_for(nblocks, 4), kThreads, 0, st>>>(packed, scales_e4m3, row_scale, nblocks,
-                                                                              bpr, (float*)y);
+    if (yt == BSQ_BF16) {
+        const int64_t nitems = rows * K / 8;
+        dequant_kernel<FMT_NV, uint16_t, 16, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
+            packed, scales_e4m3, row_scale, bpr, nitems, (uint16_t*)y);
+    } else {
+        const int64_t nitems = rows * K / 4;
+        dequant_kernel<FMT_NV, float, 16, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
+            packed, scales_e4m3, row_scale, bpr, nitems, (float*)y);
+    }
     return check_launch("bsq_dequantize_nvfp4");
 }
 
@@ -880,14 +839,18 @@ BSQ_API bsq_status bsq_dequantize_mxfp4(const uint8_t* packed, const uint8_t* sc
     BSQ_TRY(check_matrix("bsq_dequantize_mxfp4", packed, rows, K, 32));
     if (rows * K == 0) return BSQ_OK;
     if (!scales_e8m0 || !y) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_mxfp4: null pointer");
-    if (!aligned(packed, 16) || !aligned(y, 16)) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_mxfp4: misaligned pointer");
-    const int64_t nblocks = rows * K / 32;
+    if (!aligned(packed, 4) || !aligned(y, 16)) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_mxfp4: misaligned pointer");
     cudaStream_t st = (cudaStream_t)stream;
-    if (yt == BSQ_BF16)
-        mx_dequant_kernel<uint16_t, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(packed, scales_e8m0, nblocks,
-                                                                                 (uint16_t*)y);
-    else
-        mx_dequant_kernel<float, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(packed, scales_e8m0, nblocks, (float*)y);
+    const FastDiv none = make_fastdiv(1);
+    if (yt == BSQ_BF16) {
+        const int64_t nitems = rows * K / 8;
+        dequant_kernel<FMT_MX, uint16_t, 32, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
+            packed, scales_e8m0, nullptr, none, nitems, (uint16_t*)y);
+    } else {
+        const int64_t nitems = rows * K / 4;
+        dequant_kernel<FMT_MX, float, 32, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
+            packed, scales_e8m0, nullptr, none, nitems, (float*)y);
+    }
     return check_launch("bsq_dequantize_mxfp4");
 }
 
@@ -919,16 +882,16 @@ BSQ_API bsq_status bsq_dequantize_fp8(const uint8_t* codes_e4m3, const uint8_t* 
     BSQ_TRY(check_matrix("bsq_dequantize_fp8", codes_e4m3, rows, K, block));
     if (rows * K == 0) return BSQ_OK;
     if (!scales_e8m0 || !y) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_fp8: null pointer");
-    if (!aligned(codes_e4m3, 16) || !aligned(y, 16)) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_fp8: misaligned pointer");
-    const int64_t nitems = rows * K / 16;
-    const int grid = grid_for(nitems, 2);
+    if (!aligned(codes_e4m3, 8) || !aligned(y, 16)) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_fp8: misaligned pointer");
     cudaStream_t st = (cudaStream_t)stream;
+    const FastDiv none = make_fastdiv(1);
+    const int64_t nb = rows * K / 8, nf = rows * K / 4;
     if (yt == BSQ_BF16) {
-        if (block == 32) fp8_dequant_kernel<uint16_t, 32, 2><<<grid, kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nitems, (uint16_t*)y);
-        else fp8_dequant_kernel<uint16_t, 16, 2><<<grid, kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nitems, (uint16_t*)y);
+        if (block == 32) dequant_kernel<FMT_FP8, uint16_t, 32, 4><<<grid_for(nb, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nb, (uint16_t*)y);
+        else dequant_kernel<FMT_FP8, uint16_t, 16, 4><<<grid_for(nb, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nb, (uint16_t*)y);
     } else {
-        if (block == 32) fp8_dequant_kernel<float, 32, 2><<<grid, kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nitems, (float*)y);
-        else fp8_dequant_kernel<float, 16, 2><<<grid, kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nitems, (float*)y);
+        if (block == 32) dequant_kernel<FMT_FP8, float, 32, 4><<<grid_for(nf, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nf, (float*)y);
+        else dequant_kernel<FMT_FP8, float, 16, 4><<<grid_for(nf, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nf, (float*)y);
     }
     return check_launch("bsq_dequantize_fp8");
 }
