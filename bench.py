@@ -49,6 +49,8 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the sub-measurements of the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--only", default="", help="comma list of extra sections to run (nvfp4,cache,linear,gemm)")
+    ap.add_argument("--gemm-only", default="", help="time only these grouped-GEMM variants (comma list of "
+                    "mxfp4_fwd,mxfp4_bwd,nvfp4_fwd,nvfp4_bwd) and print them; for profiling")
     return ap.parse_args()
 
 
@@ -250,6 +252,14 @@ def main():
         run_reference(args)
         return
     import torch
+    if args.gemm_only:
+        from fp8_microscaling_quantization_b200 import bsq, synth
+        peaks, peak_kind = load_peaks()
+        dev = torch.device("cuda", 0)
+        res = bench_gemm(torch, bsq, synth, dev, torch.cuda.current_stream(), peaks, peak_kind,
+                         variants=set(args.gemm_only.split(",")), iters=max(1, args.steps), warm=args.warmup)
+        print(json.dumps({"grouped_gemm": res}), flush=True)
+        return
     import torch.distributed as dist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -507,7 +517,7 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
     return out
 
 
-def bench_gemm(torch, bsq, synth, dev, stream, peaks, peak_kind):
+def bench_gemm(torch, bsq, synth, dev, stream, peaks, peak_kind, variants=None, iters=10, warm=3):
     import numpy as np
     T, Kd, Nd, Ed = 16384, 7168, 2048, 32
     rng = np.random.default_rng(20260005)
@@ -517,8 +527,10 @@ def bench_gemm(torch, bsq, synth, dev, stream, peaks, peak_kind):
     x = torch.randn((T, Kd), generator=g, device=dev).to(torch.bfloat16)
     go = torch.randn((T, Nd), generator=g, device=dev).to(torch.bfloat16)
     w = (torch.randn((Ed, Nd, Kd), generator=g, device=dev) * 0.02).to(torch.bfloat16)
-    mx_p, mx_s = bsq.bsq_quantize_mxfp4(w)
-    nv_p, nv_s, nv_r = bsq.bsq_quantize_nvfp4(w)
+    want_mx = not variants or any(v.startswith("mxfp4") for v in variants)
+    want_nv = not variants or any(v.startswith("nvfp4") for v in variants)
+    mx_p, mx_s = bsq.bsq_quantize_mxfp4(w) if want_mx else (None, None)
+    nv_p, nv_s, nv_r = bsq.bsq_quantize_nvfp4(w) if want_nv else (None, None, None)
     del w
     offs = torch.from_numpy(offs_np).to(dev)
     flops = 2.0 * T * Nd * Kd
@@ -530,11 +542,13 @@ def bench_gemm(torch, bsq, synth, dev, stream, peaks, peak_kind):
     for fmt_name, fmt, p, s, r in (("mxfp4", bsq.Format.MXFP4, mx_p, mx_s, None),
                                    ("nvfp4", bsq.Format.NVFP4, nv_p, nv_s, nv_r)):
         for dname, d, a, o in (("fwd", bsq.Direction.FWD, x, out_f), ("bwd", bsq.Direction.BWD, go, out_b)):
+            if variants and f"{fmt_name}_{dname}" not in variants:
+                continue
             fn = lambda: bsq.bsq_grouped_mm_fp4(fmt, d, a, p, s, r, offs, out=o, err=err)
             t = Timer(torch, stream)
-            for _ in range(3):
+            for _ in range(warm):
                 fn()
-            for _ in range(10):
+            for _ in range(iters):
                 t.run("k", fn)
             torch.cuda.synchronize()
             ms = t.avg_ms("k")

@@ -7,24 +7,31 @@
 // shared memory as bf16, in exactly the 128-byte-swizzled layout the tensor
 // core reads, and tcgen05 MMAs accumulate fp32 in tensor memory.
 //
+// The MMA computes the transposed product, D[feature, token]: the weight tile
+// (128 output features) is the M = 128 operand A and the expert's tokens (up
+// to 256, rounded up to 16) are the N operand B.  Dequantization work per
+// tensor-core operation is set by the weight rows of a tile, so this halves it
+// against a 256-feature by 128-token tile, and a short expert pads its token
+// count only to a multiple of 16.
+//
 // Persistent, warp-specialised CTA (one per SM, 448 threads):
 //   warps 0-3   epilogue: tensor memory -> registers (x row scale for NVFP4
-//               forward) -> bf16 -> global, rows past the expert masked
-//   warps 4-11  B producers: packed weights + scales from global (two k-steps
-//               in flight), e2m1 -> bf16 via byte permutes, times the block
-//               scale (bf16x2 multiply), 16-byte swizzled shared stores
-//   warp 12     A producer: TMA loads of 128 x 64 activation tiles
+//               forward) -> bf16 -> global; lane = feature, so each store of
+//               a token's 32 features is one coalesced 64-byte row piece
+//   warps 4-11  A producers: packed weights + scales from global (several
+//               k-steps in flight), e2m1 -> bf16 by byte permutes, times the
+//               block scale (bf16x2 multiply), swizzled 16-byte shared stores
+//   warp 12     B producer: TMA loads of 64-token x 64-k activation boxes
 //   warp 13     tensor-memory allocation and the single MMA-issuing thread
-// Tile = 128 activation rows x 256 output columns, k-step 64, 4 shared-memory
-// stages; two 256-column fp32 accumulators in tensor memory so the epilogue
-// of one tile overlaps the main loop of the next.  Tiles are numbered
-// (expert m-tile, n-tile) with the n-tile fastest and dealt round-robin to the
+// Tile = 128 features x up to 256 tokens, k-step 64, 4 shared-memory stages;
+// two 256-column fp32 accumulators in tensor memory so the epilogue of one
+// tile overlaps the main loop of the next.  Tiles are numbered (expert token
+// tile, feature tile) with the feature tile fastest, dealt round-robin to the
 // CTAs; every CTA derives the tile table from offs on the device.
 //
-// Forward: B tile = 256 weight rows x 64 k (K-major operand).
-// Backward: B tile = 64 weight rows (the contraction) x 256 k (MN-major
-// operand); NVFP4's row scale lies on the contraction dimension there and is
-// folded into the dequantized bf16 weight.
+// Forward: A = 128 weight rows x 64 k (K-major).  Backward: A = W^T, 128 k
+// columns x 64 weight rows of the contraction (MN-major); NVFP4's row scale
+// lies on the contraction there and is folded into the dequantized weight.
 //
 // Every mbarrier wait gives up after about a second: the thread records
 // BSQ_DEVERR_TIMEOUT in the error word and raises a CTA-wide abort flag, all
@@ -45,20 +52,24 @@ using namespace sm100;
 
 namespace gmm {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int WM = 128;   // features per tile (MMA M)
+constexpr int TN = 256;   // tokens per tile at most (MMA N)
+constexpr int BK = 64, STAGES = 4;
+constexpr int XBOX = 64;  // token rows per TMA box
 constexpr int kEpiWarps = 4, kDqWarps = 8;
 constexpr int kTmaWarp = kEpiWarps + kDqWarps;  // 12
 constexpr int kMmaWarp = kTmaWarp + 1;          // 13
 constexpr int kThreads = (kMmaWarp + 1) * 32;   // 448
-constexpr int kDqThreads = kDqWarps * 32;       // 256
-constexpr uint32_t kAStage = BM * BK * 2;       // 16 KiB
-constexpr uint32_t kBStage = BN * BK * 2;       // 32 KiB
+constexpr uint32_t kWStage = WM * BK * 2;       // 16 KiB dequantized weights
+constexpr uint32_t kXStage = TN * BK * 2;       // 32 KiB activations
+constexpr uint32_t kXBoxBytes = XBOX * BK * 2;  // 8 KiB
 constexpr int kMaxExperts = 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr int kPrefetch = 4;  // k-steps of packed weights in flight per producer thread
 
-constexpr size_t kBarOffset = (size_t)STAGES * (kAStage + kBStage);
-constexpr int kNumBars = 3 * STAGES + 5;  // a_full, b_full, empty, acc_full[2], acc_empty[2], drain
+constexpr size_t kBarOffset = (size_t)STAGES * (kWStage + kXStage);
+constexpr int kNumBars = 3 * STAGES + 5;  // w_full, x_full, empty, acc_full[2], acc_empty[2], drain
 constexpr size_t kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 + 16 /* tmem slot, flags */ +
                               4 * (2 * kMaxExperts + 2);
 
@@ -73,40 +84,43 @@ struct Args {
 };
 
 struct Tile {
-    int e, row0, rows, n0;
+    int e;      // expert
+    int tok0;   // first token row
+    int ntok;   // tokens in the tile (1..256)
+    int f0;     // first feature (output column) of the tile
 };
 
 struct Shared {
-    uint8_t* a;
-    uint8_t* b;
-    uint64_t* a_full;
-    uint64_t* b_full;
+    uint8_t* w;
+    uint8_t* x;
+    uint64_t* w_full;
+    uint64_t* x_full;
     uint64_t* empty;
     uint64_t* acc_full;
     uint64_t* acc_empty;
     uint64_t* drain;
     uint32_t* tmem_slot;
     volatile int* abort;
-    int* mt_prefix;  // [E + 1] first m-tile of each expert
+    int* tt_prefix;  // [E + 1] first token tile of each expert
     int* seg;        // [E + 1] seg[e] = first row of expert e, seg[E] = offs[E-1]
 };
 
 __device__ __forceinline__ Shared carve(uint8_t* raw) {
     Shared s;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-    s.a = base;
-    s.b = base + STAGES * kAStage;
+    s.w = base;
+    s.x = base + STAGES * kWStage;
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + kBarOffset);
-    s.a_full = bars;
-    s.b_full = bars + STAGES;
+    s.w_full = bars;
+    s.x_full = bars + STAGES;
     s.empty = bars + 2 * STAGES;
     s.acc_full = bars + 3 * STAGES;
     s.acc_empty = s.acc_full + 2;
     s.drain = s.acc_empty + 2;
     s.tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
     s.abort = reinterpret_cast<volatile int*>(s.tmem_slot + 1);
-    s.mt_prefix = reinterpret_cast<int*>(s.tmem_slot + 4);
-    s.seg = s.mt_prefix + kMaxExperts + 1;
+    s.tt_prefix = reinterpret_cast<int*>(s.tmem_slot + 4);
+    s.seg = s.tt_prefix + kMaxExperts + 1;
     return s;
 }
 
@@ -125,20 +139,20 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const S
     return true;
 }
 
-__device__ __forceinline__ Tile decode_tile(int t, int n_tiles, int E, const Shared& sh) {
-    const int mg = t / n_tiles;
-    const int nt = t - mg * n_tiles;
-    int lo = 0, hi = E - 1;  // last expert whose first m-tile is <= mg
+__device__ __forceinline__ Tile decode_tile(int t, int f_tiles, int E, const Shared& sh) {
+    const int tg = t / f_tiles;
+    const int ft = t - tg * f_tiles;
+    int lo = 0, hi = E - 1;  // last expert whose first token tile is <= tg
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (sh.mt_prefix[mid] <= mg) lo = mid;
+        if (sh.tt_prefix[mid] <= tg) lo = mid;
         else hi = mid - 1;
     }
     Tile ti;
     ti.e = lo;
-    ti.row0 = sh.seg[lo] + (mg - sh.mt_prefix[lo]) * BM;
-    ti.rows = min(BM, sh.seg[lo + 1] - ti.row0);
-    ti.n0 = nt * BN;
+    ti.tok0 = sh.seg[lo] + (tg - sh.tt_prefix[lo]) * TN;
+    ti.ntok = min(TN, sh.seg[lo + 1] - ti.tok0);
+    ti.f0 = ft * WM;
     return ti;
 }
 
@@ -189,26 +203,31 @@ __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t code, float g) {
     return b | (b << 16);
 }
 
+// One producer thread's share of a k-step: 32 consecutive packed weights.
 struct Unit {
     uint4 pk;
     uint32_t sc;  // MXFP4: one e8m0 byte; NVFP4: two e4m3 bytes (16-column halves)
     float g;      // NVFP4 backward row scale
 };
 
+// Forward: unit u = (feature row u/2 of the tile, k half u%2).  Backward:
+// unit u = (contraction row u/4 of the k-step, 32-column segment u%4 of the
+// tile's 128 k columns).
 template <int FMT, int DIR>
 __device__ __forceinline__ void load_unit(Unit& u, const Args& a, const Tile& ti, int ks, int unit) {
     int64_t row;
     int kcol;  // first weight column (k) of the unit's 32 elements
     if (DIR == BSQ_FWD) {
-        row = (int64_t)ti.e * a.N + ti.n0 + (unit >> 1);
+        row = (int64_t)ti.e * a.N + ti.f0 + (unit >> 1);
         kcol = ks * BK + (unit & 1) * 32;
     } else {
-        row = (int64_t)ti.e * a.N + ks * BK + (unit >> 3);
-        kcol = ti.n0 + (unit & 7) * 32;
+        row = (int64_t)ti.e * a.N + ks * BK + (unit >> 2);
+        kcol = ti.f0 + (unit & 3) * 32;
     }
     u.pk = __ldg(reinterpret_cast<const uint4*>(a.packed + row * (a.K / 2) + kcol / 2));
     if (FMT == BSQ_MXFP4) {
         u.sc = __ldg(a.scales + row * (a.K / 32) + kcol / 32);
+        u.g = 1.0f;
     } else {
         u.sc = __ldg(reinterpret_cast<const unsigned short*>(a.scales + row * (a.K / 16) + kcol / 16));
         u.g = (DIR == BSQ_BWD) ? __ldg(a.row_scale + row) : 1.0f;
@@ -216,7 +235,7 @@ __device__ __forceinline__ void load_unit(Unit& u, const Args& a, const Tile& ti
 }
 
 template <int FMT, int DIR>
-__device__ __forceinline__ void store_unit(const Unit& u, uint32_t b_stage, int unit) {
+__device__ __forceinline__ void store_unit(const Unit& u, uint32_t w_stage, int unit) {
     uint32_t s_lo, s_hi;
     if (FMT == BSQ_MXFP4) {
         s_lo = s_hi = scale_bf16x2<FMT, false>(u.sc, 0.0f);
@@ -224,45 +243,45 @@ __device__ __forceinline__ void store_unit(const Unit& u, uint32_t b_stage, int 
         s_lo = scale_bf16x2<FMT, DIR == BSQ_BWD>(u.sc & 0xFFu, u.g);
         s_hi = scale_bf16x2<FMT, DIR == BSQ_BWD>(u.sc >> 8, u.g);
     }
-    // smem row and first 16-byte chunk of this unit inside the 128-byte row
+    // 128-byte shared row of the unit and its first 16-byte chunk in that row
     uint32_t base;
     int r, c0;
     if (DIR == BSQ_FWD) {
-        r = unit >> 1;
+        r = unit >> 1;  // K-major: one row per feature, 8-row atoms of 1 KiB
         c0 = (unit & 1) * 4;
-        base = b_stage + (r >> 3) * 1024 + (r & 7) * 128;
+        base = w_stage + (r >> 3) * 1024 + (r & 7) * 128;
     } else {
-        r = unit >> 3;
-        const int seg = unit & 7;
+        r = unit >> 2;  // MN-major: one row per contraction index, 64-feature panels
+        const int seg = unit & 3;
         c0 = (seg & 1) * 4;
-        base = b_stage + (seg >> 1) * (BK * 128) + (r >> 3) * 1024 + (r & 7) * 128;
+        base = w_stage + (seg >> 1) * (BK * 128) + (r >> 3) * 1024 + (r & 7) * 128;
     }
     const uint32_t words[4] = {u.pk.x, u.pk.y, u.pk.z, u.pk.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         uint32_t v[4];
         e2m1x8_to_bf16(words[i], v);
-        const uint32_t s = (i < 2) ? s_lo : s_hi;
+        const uint32_t sc = (i < 2) ? s_lo : s_hi;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = mul_bf16x2(v[j], s);
+        for (int j = 0; j < 4; ++j) v[j] = mul_bf16x2(v[j], sc);
         sts128(base + (uint32_t)(((c0 + i) ^ (r & 7)) << 4), v[0], v[1], v[2], v[3]);
     }
 }
 
 template <int FMT, int DIR>
-__global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_constant__ CUtensorMap tmap_a, Args args) {
+__global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_constant__ CUtensorMap tmap_x, Args args) {
     extern __shared__ uint8_t smem_raw[];
     const Shared sh = carve(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = args.E;
-    const int n_tiles = (DIR == BSQ_FWD ? args.N : args.K) / BN;
+    const int f_tiles = (DIR == BSQ_FWD ? args.N : args.K) / WM;
     const int k_steps = (DIR == BSQ_FWD ? args.K : args.N) / BK;
     const int out_w = (DIR == BSQ_FWD ? args.N : args.K);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&sh.a_full[s], 1);
-            mbar_init(&sh.b_full[s], kDqThreads);
+            mbar_init(&sh.w_full[s], kDqWarps);
+            mbar_init(&sh.x_full[s], 1);
             mbar_init(&sh.empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -277,13 +296,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
             const int o = args.offs[e];
             if (o < prev || o > args.T) bad = 1;
             sh.seg[e] = prev;
-            sh.mt_prefix[e] = total;
-            const int cnt = o - prev;
-            if (!bad) total += (cnt + BM - 1) / BM;
+            sh.tt_prefix[e] = total;
+            if (!bad) total += (o - prev + TN - 1) / TN;
             prev = o;
         }
         sh.seg[E] = bad ? 0 : prev;
-        sh.mt_prefix[E] = total;
+        sh.tt_prefix[E] = total;
         sh.tmem_slot[1] = 0;  // abort flag
         sh.tmem_slot[2] = bad;
         sh.tmem_slot[3] = bad ? 0 : total;
@@ -293,13 +311,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
         tmem_alloc(sh.tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (warp == kTmaWarp && lane == 0) tma_prefetch_desc(&tmap_a);
+    if (warp == kTmaWarp && lane == 0) tma_prefetch_desc(&tmap_x);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_slot[0];
     const int bad = sh.tmem_slot[2];
-    const int num_tiles = bad ? 0 : sh.tmem_slot[3] * n_tiles;
+    const int num_tiles = bad ? 0 : sh.tmem_slot[3] * f_tiles;
 
     if (warp < kEpiWarps) {
         // ---------------------------------------------------------- epilogue
@@ -312,44 +330,32 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                 for (int v = tid; v < vec_per_row; v += kEpiWarps * 32) dst[v] = make_uint4(0, 0, 0, 0);
             }
         }
-        const int q = warp;  // tensor-memory lane quadrant of this warp
+        const int q = warp;  // tensor-memory lane quadrant of this warp = features 32q..32q+31
         int tile_iter = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tile_iter) {
-            const Tile ti = decode_tile(t, n_tiles, E, sh);
+            const Tile ti = decode_tile(t, f_tiles, E, sh);
             const int acc = tile_iter & 1;
             if (!wait_bar(&sh.acc_full[acc], (tile_iter >> 1) & 1, sh, args.err)) break;
             tc_fence_after();
-            const int rit = q * 32 + lane;
-            const bool valid = rit < ti.rows;
-            uint16_t* orow = args.out + (int64_t)(ti.row0 + rit) * out_w + ti.n0;
-            const float* grow = (FMT == BSQ_NVFP4 && DIR == BSQ_FWD)
-                                    ? args.row_scale + (int64_t)ti.e * args.N + ti.n0 : nullptr;
+            const int f = ti.f0 + q * 32 + lane;
+            float gf = 1.0f;
+            if (FMT == BSQ_NVFP4 && DIR == BSQ_FWD) gf = __ldg(args.row_scale + (int64_t)ti.e * args.N + f);
+            uint16_t* ocol = args.out + (int64_t)ti.tok0 * out_w + f;
+            const int chunks = (ti.ntok + 15) >> 4;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c * 32), r);
+            for (int c = 0; c < chunks; ++c) {
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TN + c * 16), r);
                 tmem_ld_wait();
-                float f[32];
+                const int nv = min(16, ti.ntok - c * 16);
+                uint16_t* p = ocol + (int64_t)(c * 16) * out_w;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(r[j]);
-                if (FMT == BSQ_NVFP4 && DIR == BSQ_FWD) {
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        const float4 g4 = __ldg(reinterpret_cast<const float4*>(grow + c * 32 + j));
-                        f[j] *= g4.x; f[j + 1] *= g4.y; f[j + 2] *= g4.z; f[j + 3] *= g4.w;
-                    }
-                }
-                if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint4 o;
-                        o.x = pack_bf16x2(f[8 * v + 0], f[8 * v + 1]);
-                        o.y = pack_bf16x2(f[8 * v + 2], f[8 * v + 3]);
-                        o.z = pack_bf16x2(f[8 * v + 4], f[8 * v + 5]);
-                        o.w = pack_bf16x2(f[8 * v + 6], f[8 * v + 7]);
-                        dst[v] = o;
-                    }
+                for (int j = 0; j < 16; ++j) {
+                    float v = __uint_as_float(r[j]);
+                    if (FMT == BSQ_NVFP4 && DIR == BSQ_FWD) v *= gf;
+                    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+                    if (j < nv) *p = *reinterpret_cast<const uint16_t*>(&h);
+                    p += out_w;
                 }
             }
             tc_fence_before();
@@ -357,105 +363,108 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
             if (lane == 0) mbar_arrive(&sh.acc_empty[acc]);
         }
     } else if (warp < kTmaWarp) {
-        // ------------------------------------------------------- B producers
-        const int dq = threadIdx.x - kEpiWarps * 32;  // 0..255
-        const uint32_t b_base = smem_u32(sh.b);
+        // ------------------------------------------------- A (weight) producers
+        const int dq = threadIdx.x - kEpiWarps * 32;  // 0..255 = unit index
+        const uint32_t w_base = smem_u32(sh.w);
         int my_tiles = 0;
         if (num_tiles > (int)blockIdx.x) my_tiles = (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1;
         const int items = my_tiles * k_steps;
-        // load cursor (runs two items ahead of the stores)
+        // load cursor, kPrefetch k-steps ahead of the stores
         int lt = blockIdx.x, lks = 0;
         Tile lti;
-        if (items > 0) lti = decode_tile(lt, n_tiles, E, sh);
-        Unit buf[2][2];
-        auto advance = [&]() {
-            if (++lks == k_steps) {
-                lks = 0;
-                lt += gridDim.x;
-                if (lt < num_tiles) lti = decode_tile(lt, n_tiles, E, sh);
-            }
-        };
+        if (items > 0) lti = decode_tile(lt, f_tiles, E, sh);
+        Unit buf[kPrefetch];
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < kPrefetch; ++b) {
             if (b < items) {
-                load_unit<FMT, DIR>(buf[b][0], args, lti, lks, dq);
-                load_unit<FMT, DIR>(buf[b][1], args, lti, lks, dq + kDqThreads);
-                advance();
+                load_unit<FMT, DIR>(buf[b], args, lti, lks, dq);
+                if (++lks == k_steps) {
+                    lks = 0;
+                    lt += gridDim.x;
+                    if (lt < num_tiles) lti = decode_tile(lt, f_tiles, E, sh);
+                }
             }
         }
         bool ok = true;
-        for (int it = 0; it < items && ok; it += 2) {
+        for (int it = 0; it < items && ok; it += kPrefetch) {
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
+            for (int b = 0; b < kPrefetch; ++b) {
                 const int i = it + b;
                 if (i < items && ok) {
                     const int s = i % STAGES;
                     if (!wait_bar(&sh.empty[s], ((i / STAGES) & 1) ^ 1, sh, args.err)) {
                         ok = false;
                     } else {
-                        const uint32_t stage = b_base + s * kBStage;
-                        store_unit<FMT, DIR>(buf[b][0], stage, dq);
-                        store_unit<FMT, DIR>(buf[b][1], stage, dq + kDqThreads);
+                        store_unit<FMT, DIR>(buf[b], w_base + s * kWStage, dq);
                         fence_proxy_async_smem();
-                        mbar_arrive(&sh.b_full[s]);
-                        if (i + 2 < items) {
-                            load_unit<FMT, DIR>(buf[b][0], args, lti, lks, dq);
-                            load_unit<FMT, DIR>(buf[b][1], args, lti, lks, dq + kDqThreads);
-                            advance();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sh.w_full[s]);
+                        if (i + kPrefetch < items) {
+                            load_unit<FMT, DIR>(buf[b], args, lti, lks, dq);
+                            if (++lks == k_steps) {
+                                lks = 0;
+                                lt += gridDim.x;
+                                if (lt < num_tiles) lti = decode_tile(lt, f_tiles, E, sh);
+                            }
                         }
                     }
                 }
             }
         }
     } else if (warp == kTmaWarp) {
-        // ------------------------------------------------------- A producer
+        // ------------------------------------------- B (activation) producer
         if (lane == 0) {
             int it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                const Tile ti = decode_tile(t, n_tiles, E, sh);
+                const Tile ti = decode_tile(t, f_tiles, E, sh);
+                const int nbox = (ti.ntok + XBOX - 1) / XBOX;
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
                     const int s = it % STAGES;
                     if (!wait_bar(&sh.empty[s], ((it / STAGES) & 1) ^ 1, sh, args.err)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&sh.a_full[s], kAStage);
-                    tma_load_2d(sh.a + s * kAStage, &tmap_a, &sh.a_full[s], ks * BK, ti.row0);
+                    mbar_arrive_expect_tx(&sh.x_full[s], nbox * kXBoxBytes);
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d(sh.x + s * kXStage + b * kXBoxBytes, &tmap_x, &sh.x_full[s], ks * BK,
+                                    ti.tok0 + b * XBOX);
                 }
             }
             if (!ok) {
                 // drain the loads still in flight into this CTA's shared memory
                 for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-                    mbar_wait(&sh.a_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
+                    mbar_wait(&sh.x_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
             }
         }
     } else {
         // ----------------------------------------------------------- MMA
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(BM, BN, DIR == BSQ_BWD ? 1u : 0u);
-            const uint32_t a_base = smem_u32(sh.a), b_base = smem_u32(sh.b);
+            const uint32_t w_base = smem_u32(sh.w), x_base = smem_u32(sh.x);
             int it = 0, tile_iter = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tile_iter) {
+                const Tile ti = decode_tile(t, f_tiles, E, sh);
+                const uint32_t n_mma = (uint32_t)((ti.ntok + 15) & ~15);
+                const uint32_t idesc = idesc_bf16_ab(WM, n_mma, DIR == BSQ_BWD ? 1u : 0u, 0u);
                 const int acc = tile_iter & 1;
                 if (!wait_bar(&sh.acc_empty[acc], ((tile_iter >> 1) & 1) ^ 1, sh, args.err)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(acc * BN);
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * TN);
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!wait_bar(&sh.a_full[s], ph, sh, args.err) || !wait_bar(&sh.b_full[s], ph, sh, args.err)) {
+                    if (!wait_bar(&sh.w_full[s], ph, sh, args.err) || !wait_bar(&sh.x_full[s], ph, sh, args.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t as = a_base + s * kAStage, bs = b_base + s * kBStage;
+                    const uint32_t ws = w_base + s * kWStage, xs = x_base + s * kXStage;
 #pragma unroll
                     for (int k16 = 0; k16 < BK / 16; ++k16) {
-                        const uint64_t ad = smem_desc(as + k16 * 32, 16, 1024);
-                        const uint64_t bd = (DIR == BSQ_FWD) ? smem_desc(bs + k16 * 32, 16, 1024)
-                                                             : smem_desc(bs + k16 * 2048, BK * 128, 1024);
+                        const uint64_t ad = (DIR == BSQ_FWD) ? smem_desc(ws + k16 * 32, 16, 1024)
+                                                             : smem_desc(ws + k16 * 2048, BK * 128, 1024);
+                        const uint64_t bd = smem_desc(xs + k16 * 32, 16, 1024);
                         mma_bf16_ss(d_tmem, ad, bd, idesc, (ks | k16) != 0 ? 1u : 0u);
                     }
                     mma_commit(&sh.empty[s]);
@@ -538,8 +547,8 @@ BSQ_API bsq_status bsq_grouped_mm_fp4(bsq_format fmt, bsq_dir dir, const void* a
     if (T > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30) || (int64_t)E * N > (int64_t(1) << 31))
         return fail(BSQ_ERR_UNSUPPORTED, "%s: sizes too large", fn);
     const int64_t out_w = (dir == BSQ_FWD) ? N : K, contr = (dir == BSQ_FWD) ? K : N;
-    if (out_w % gmm::BN != 0 || contr % gmm::BK != 0 || K % 64 != 0)
-        return fail(BSQ_ERR_UNSUPPORTED, "%s: needs the output width %% %d == 0 and K, N %% %d == 0", fn, gmm::BN,
+    if (out_w % gmm::WM != 0 || contr % gmm::BK != 0 || K % 64 != 0 || N % 64 != 0)
+        return fail(BSQ_ERR_UNSUPPORTED, "%s: needs the output width %% %d == 0 and K, N %% %d == 0", fn, gmm::WM,
                     gmm::BK);
     if (!err) return fail(BSQ_ERR_INVALID_ARG, "%s: null error word", fn);
     if (T == 0) return BSQ_OK;
@@ -555,7 +564,7 @@ BSQ_API bsq_status bsq_grouped_mm_fp4(bsq_format fmt, bsq_dir dir, const void* a
     CUtensorMap tmap;
     const cuuint64_t dims[2] = {(cuuint64_t)contr, (cuuint64_t)T};
     const cuuint64_t strides[1] = {(cuuint64_t)contr * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)gmm::BK, (cuuint32_t)gmm::BM};
+    const cuuint32_t box[2] = {(cuuint32_t)gmm::BK, (cuuint32_t)gmm::XBOX};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -573,8 +582,8 @@ BSQ_API bsq_status bsq_grouped_mm_fp4(bsq_format fmt, bsq_dir dir, const void* a
     args.T = (int)T;
     args.N = (int)N;
     args.K = (int)K;
-    const int64_t n_tiles = out_w / gmm::BN;
-    const int64_t max_tiles = ((T + gmm::BM - 1) / gmm::BM + E) * n_tiles;
+    const int64_t f_tiles = out_w / gmm::WM;
+    const int64_t max_tiles = ((T + gmm::TN - 1) / gmm::TN + E) * f_tiles;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, sm_count()));
     cudaStream_t s = (cudaStream_t)stream;
     if (fmt == BSQ_MXFP4)

@@ -179,10 +179,10 @@ bsq_status bsq_quantize_cache_backward(const void* grad_out, void* grad_in, bsq_
  *   err         device uint32 word; the caller zeroes it before the call and
  *               reads it after synchronising: BSQ_DEVERR_* bits.  With a bad
  *               offs the output is undefined.
- * Rows at or past offs[E-1] are written as zero.  Requirements:
- * N % 256 == 0 for BSQ_FWD and K % 256 == 0 for BSQ_BWD (the output tile
- * width); K % 64 == 0 and N % 64 == 0 (contraction tiles); x, packed and out
- * 16-byte aligned.  Other shapes return BSQ_ERR_UNSUPPORTED. */
+ * Rows at or past offs[E-1] are written as zero.  Requirements: the output
+ * width (N for BSQ_FWD, K for BSQ_BWD) a multiple of 128 and K, N multiples
+ * of 64; E <= 1024; a, packed, out and row_scale 16-byte aligned.  Other
+ * shapes return BSQ_ERR_UNSUPPORTED. */
 bsq_status bsq_grouped_mm_fp4(bsq_format fmt, bsq_dir dir, const void* a, const uint8_t* packed,
                               const uint8_t* scales, const float* row_scale, const int32_t* offs,
                               int E, int64_t T, int64_t N, int64_t K, void* out, uint32_t* err,
