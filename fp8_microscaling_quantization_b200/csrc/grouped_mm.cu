@@ -234,8 +234,9 @@ __device__ __forceinline__ void load_unit(Unit& u, const Args& a, const Tile& ti
     }
 }
 
+// Decode a unit into 16 words of bf16x2 (four 16-byte chunks), block scale applied.
 template <int FMT, int DIR>
-__device__ __forceinline__ void store_unit(const Unit& u, uint32_t w_stage, int unit) {
+__device__ __forceinline__ void decode_unit(const Unit& u, uint32_t (&v)[16]) {
     uint32_t s_lo, s_hi;
     if (FMT == BSQ_MXFP4) {
         s_lo = s_hi = scale_bf16x2<FMT, false>(u.sc, 0.0f);
@@ -243,6 +244,20 @@ __device__ __forceinline__ void store_unit(const Unit& u, uint32_t w_stage, int 
         s_lo = scale_bf16x2<FMT, DIR == BSQ_BWD>(u.sc & 0xFFu, u.g);
         s_hi = scale_bf16x2<FMT, DIR == BSQ_BWD>(u.sc >> 8, u.g);
     }
+    const uint32_t words[4] = {u.pk.x, u.pk.y, u.pk.z, u.pk.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t t[4];
+        e2m1x8_to_bf16(words[i], t);
+        const uint32_t sc = (i < 2) ? s_lo : s_hi;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[4 * i + j] = mul_bf16x2(t[j], sc);
+    }
+}
+
+// Write the decoded unit to its place in the swizzled operand tile.
+template <int DIR>
+__device__ __forceinline__ void store_unit(const uint32_t (&v)[16], uint32_t w_stage, int unit) {
     // 128-byte shared row of the unit and its first 16-byte chunk in that row
     uint32_t base;
     int r, c0;
@@ -256,16 +271,9 @@ __device__ __forceinline__ void store_unit(const Unit& u, uint32_t w_stage, int 
         c0 = (seg & 1) * 4;
         base = w_stage + (seg >> 1) * (BK * 128) + (r >> 3) * 1024 + (r & 7) * 128;
     }
-    const uint32_t words[4] = {u.pk.x, u.pk.y, u.pk.z, u.pk.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint32_t v[4];
-        e2m1x8_to_bf16(words[i], v);
-        const uint32_t sc = (i < 2) ? s_lo : s_hi;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = mul_bf16x2(v[j], sc);
-        sts128(base + (uint32_t)(((c0 + i) ^ (r & 7)) << 4), v[0], v[1], v[2], v[3]);
-    }
+    for (int i = 0; i < 4; ++i)
+        sts128(base + (uint32_t)(((c0 + i) ^ (r & 7)) << 4), v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
 
 template <int FMT, int DIR>
@@ -391,22 +399,26 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
             for (int b = 0; b < kPrefetch; ++b) {
                 const int i = it + b;
                 if (i < items && ok) {
+                    // decode first (off the critical path), refill the buffer, then
+                    // wait for the shared-memory slot and only store + signal
+                    uint32_t v[16];
+                    decode_unit<FMT, DIR>(buf[b], v);
+                    if (i + kPrefetch < items) {
+                        load_unit<FMT, DIR>(buf[b], args, lti, lks, dq);
+                        if (++lks == k_steps) {
+                            lks = 0;
+                            lt += gridDim.x;
+                            if (lt < num_tiles) lti = decode_tile(lt, f_tiles, E, sh);
+                        }
+                    }
                     const int s = i % STAGES;
                     if (!wait_bar(&sh.empty[s], ((i / STAGES) & 1) ^ 1, sh, args.err)) {
                         ok = false;
                     } else {
-                        store_unit<FMT, DIR>(buf[b], w_base + s * kWStage, dq);
+                        store_unit<DIR>(v, w_base + s * kWStage, dq);
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&sh.w_full[s]);
-                        if (i + kPrefetch < items) {
-                            load_unit<FMT, DIR>(buf[b], args, lti, lks, dq);
-                            if (++lks == k_steps) {
-                                lks = 0;
-                                lt += gridDim.x;
-                                if (lt < num_tiles) lti = decode_tile(lt, f_tiles, E, sh);
-                            }
-                        }
                     }
                 }
             }
