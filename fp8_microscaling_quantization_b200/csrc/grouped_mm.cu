@@ -23,7 +23,8 @@
 //               block scale (bf16x2 multiply), swizzled 16-byte shared stores
 //   warp 12     B producer: TMA loads of 64-token x 64-k activation boxes
 //   warp 13     tensor-memory allocation and the single MMA-issuing thread
-// Tile = 128 features x up to 256 tokens, k-step 64, 4 shared-memory stages;
+// Tile = 128 features x up to 256 tokens, k-step 64; separate rings of 5
+// dequantized-weight slots (16 KiB) and 4 activation slots (32 KiB);
 // two 256-column fp32 accumulators in tensor memory so the epilogue of one
 // tile overlaps the main loop of the next.  Tiles are numbered (expert token
 // tile, feature tile) with the feature tile fastest, dealt round-robin to the
@@ -54,7 +55,9 @@ namespace gmm {
 
 constexpr int WM = 128;   // features per tile (MMA M)
 constexpr int TN = 256;   // tokens per tile at most (MMA N)
-constexpr int BK = 64, STAGES = 4;
+constexpr int BK = 64;
+constexpr int WSTAGES = 5;  // dequantized-weight ring (16 KiB slots)
+constexpr int XSTAGES = 4;  // activation ring (32 KiB slots)
 constexpr int XBOX = 64;  // token rows per TMA box
 constexpr int kEpiWarps = 4, kDqWarps = 8;
 constexpr int kTmaWarp = kEpiWarps + kDqWarps;  // 12
@@ -68,8 +71,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kPrefetch = 4;  // k-steps of packed weights in flight per producer thread
 
-constexpr size_t kBarOffset = (size_t)STAGES * (kWStage + kXStage);
-constexpr int kNumBars = 3 * STAGES + 5;  // w_full, x_full, empty, acc_full[2], acc_empty[2], drain
+constexpr size_t kBarOffset = (size_t)WSTAGES * kWStage + (size_t)XSTAGES * kXStage;
+constexpr int kNumBars = 2 * WSTAGES + 2 * XSTAGES + 5;  // w_full/empty, x_full/empty, acc_full[2], acc_empty[2], drain
 constexpr size_t kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 + 16 /* tmem slot, flags */ +
                               4 * (2 * kMaxExperts + 2);
 
@@ -94,8 +97,9 @@ struct Shared {
     uint8_t* w;
     uint8_t* x;
     uint64_t* w_full;
+    uint64_t* w_empty;
     uint64_t* x_full;
-    uint64_t* empty;
+    uint64_t* x_empty;
     uint64_t* acc_full;
     uint64_t* acc_empty;
     uint64_t* drain;
@@ -109,12 +113,13 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
     Shared s;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     s.w = base;
-    s.x = base + STAGES * kWStage;
+    s.x = base + WSTAGES * kWStage;
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + kBarOffset);
     s.w_full = bars;
-    s.x_full = bars + STAGES;
-    s.empty = bars + 2 * STAGES;
-    s.acc_full = bars + 3 * STAGES;
+    s.w_empty = bars + WSTAGES;
+    s.x_full = bars + 2 * WSTAGES;
+    s.x_empty = bars + 2 * WSTAGES + XSTAGES;
+    s.acc_full = bars + 2 * WSTAGES + 2 * XSTAGES;
     s.acc_empty = s.acc_full + 2;
     s.drain = s.acc_empty + 2;
     s.tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
@@ -287,10 +292,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
     const int out_w = (DIR == BSQ_FWD ? args.N : args.K);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < WSTAGES; ++s) {
             mbar_init(&sh.w_full[s], kDqWarps);
+            mbar_init(&sh.w_empty[s], 1);
+        }
+        for (int s = 0; s < XSTAGES; ++s) {
             mbar_init(&sh.x_full[s], 1);
-            mbar_init(&sh.empty[s], 1);
+            mbar_init(&sh.x_empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sh.acc_full[i], 1);
@@ -411,8 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                             if (lt < num_tiles) lti = decode_tile(lt, f_tiles, E, sh);
                         }
                     }
-                    const int s = i % STAGES;
-                    if (!wait_bar(&sh.empty[s], ((i / STAGES) & 1) ^ 1, sh, args.err)) {
+                    const int s = i % WSTAGES;
+                    if (!wait_bar(&sh.w_empty[s], ((i / WSTAGES) & 1) ^ 1, sh, args.err)) {
                         ok = false;
                     } else {
                         store_unit<DIR>(v, w_base + s * kWStage, dq);
@@ -432,8 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                 const Tile ti = decode_tile(t, f_tiles, E, sh);
                 const int nbox = (ti.ntok + XBOX - 1) / XBOX;
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
-                    const int s = it % STAGES;
-                    if (!wait_bar(&sh.empty[s], ((it / STAGES) & 1) ^ 1, sh, args.err)) {
+                    const int s = it % XSTAGES;
+                    if (!wait_bar(&sh.x_empty[s], ((it / XSTAGES) & 1) ^ 1, sh, args.err)) {
                         ok = false;
                         break;
                     }
@@ -445,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
             }
             if (!ok) {
                 // drain the loads still in flight into this CTA's shared memory
-                for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-                    mbar_wait(&sh.x_full[j % STAGES], (j / STAGES) & 1, kWaitNs);
+                for (int j = (it > XSTAGES ? it - XSTAGES : 0); j < it; ++j)
+                    mbar_wait(&sh.x_full[j % XSTAGES], (j / XSTAGES) & 1, kWaitNs);
             }
         }
     } else {
@@ -464,14 +472,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * TN);
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
-                    if (!wait_bar(&sh.w_full[s], ph, sh, args.err) || !wait_bar(&sh.x_full[s], ph, sh, args.err)) {
+                    const int sw = it % WSTAGES, sx = it % XSTAGES;
+                    if (!wait_bar(&sh.w_full[sw], (it / WSTAGES) & 1, sh, args.err) ||
+                        !wait_bar(&sh.x_full[sx], (it / XSTAGES) & 1, sh, args.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t ws = w_base + s * kWStage, xs = x_base + s * kXStage;
+                    const uint32_t ws = w_base + sw * kWStage, xs = x_base + sx * kXStage;
 #pragma unroll
                     for (int k16 = 0; k16 < BK / 16; ++k16) {
                         const uint64_t ad = (DIR == BSQ_FWD) ? smem_desc(ws + k16 * 32, 16, 1024)
@@ -479,7 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                         const uint64_t bd = smem_desc(xs + k16 * 32, 16, 1024);
                         mma_bf16_ss(d_tmem, ad, bd, idesc, (ks | k16) != 0 ? 1u : 0u);
                     }
-                    mma_commit(&sh.empty[s]);
+                    mma_commit(&sh.w_empty[sw]);
+                    mma_commit(&sh.x_empty[sx]);
                 }
                 if (ok) mma_commit(&sh.acc_full[acc]);
             }
