@@ -64,30 +64,36 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash():
+KERNEL_SOURCES = {
+    "quant": ["quant.cu", "formats.cuh", "host_util.h"],
+    "gemm": ["grouped_mm.cu", "tcgen05.cuh", "formats.cuh", "host_util.h"],
+}
+
+
+def kernel_source_hash(family):
+    """Hash of the source files a kernel family is built from (a committed
+    ncu traffic figure is only reported while it matches)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp8_microscaling_quantization_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in KERNEL_SOURCES[family]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def traffic_from_profiles(kernel_key):
-    """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None
-    if the summary is missing or was taken on different kernel sources."""
+def traffic_from_profiles(kernel_key, family="quant"):
+    """Per-launch DRAM bytes (read + write) of a kernel from the committed ncu
+    summary profiles/dram_traffic.json, or None if it is missing or was taken
+    on different kernel sources."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
     except Exception:
         return None
-    if d.get("source_hash") != kernel_source_hash():
-        return None
     ent = d.get("kernels", {}).get(kernel_key)
-    if not ent:
+    if not ent or ent.get("source_hash") != kernel_source_hash(family):
         return None
     return ent.get("bytes_per_launch")
 

@@ -21,6 +21,7 @@
 
 #include "formats.cuh"
 #include "host_util.h"
+#include "tcgen05.cuh"
 
 namespace bsq {
 
@@ -225,6 +226,36 @@ __device__ __forceinline__ void build_e2m1_lut(float2* lut) {
 // Quantize one 8-element chunk whose block partner is lane ^ 1, given the
 // row scale g (g == 0: zero row).  Returns the packed 4 bytes; *scale_byte
 // receives the block's e4m3 scale.
+// e2m1 codes of RN(v[j] / d) for 8 values, bit-exact, mostly without a
+// division.  With r = RN(1/d), q = RN(v * r) lies within 1.5 * 2**-23 * |q| of
+// RN(v / d) (two roundings of 2**-24 each, d and r normal).  The e2m1 rounding
+// is monotone in |q|, so if the two brackets q * (1 - 2**-21) and
+// q * (1 + 2**-21), which enclose RN(v / d), round to the same codes, those
+// are the codes of RN(v / d); only when a bracket straddles a rounding
+// boundary (rare) or d is out of range is the quotient computed by IEEE
+// division.
+__device__ __forceinline__ uint32_t e2m1x8_of_quotient(const float v[8], float d) {
+    if (d >= 2.3509887e-38f /* 2**-125 */ && d <= 4.2535296e37f /* 2**125 */) {
+        const float r = __frcp_rn(d);
+        float lo[8], hi[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float q = __fmul_rn(v[j], r);
+            lo[j] = __fmul_rn(q, 0.99999952f);  // 1 - 2**-21
+            hi[j] = __fmul_rn(q, 1.00000048f);  // 1 + 2**-21
+        }
+        const uint32_t clo = e2m1x8_encode_hw(lo), chi = e2m1x8_encode_hw(hi);
+        if (clo == chi) return clo;
+    }
+    float q[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) q[j] = __fdiv_rn(v[j], d);
+    return e2m1x8_encode_hw(q);
+}
+
+// Quantize one 8-element chunk whose block partner is lane ^ 1, given the
+// row scale g (g == 0: zero row).  Returns the packed 4 bytes; *scale_byte
+// receives the block's e4m3 scale.
 __device__ __forceinline__ uint32_t nv_quant_chunk(const float v[8], float g, uint32_t* scale_byte) {
     const float amax_b = group_max<2>(amax8(v));
     if (g == 0.0f) {
@@ -233,70 +264,81 @@ __device__ __forceinline__ uint32_t nv_quant_chunk(const float v[8], float g, ui
     }
     const uint32_t s = nv_scale_byte(amax_b, g);
     const float d = __fmul_rn(e4m3_decode(s), g);
-    float q[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) q[j] = __fdiv_rn(v[j], d);
     *scale_byte = s;
-    return e2m1x8_encode_hw(q);
+    return e2m1x8_of_quotient(v, d);
 }
 
-// Per-row amax rule: one CTA per row (grid-stride over rows); the row stays in
-// registers (NCH chunks per thread) between the amax and the quantization.
-template <typename T, int NCH>
+// Per-row amax rule: one CTA per row (grid-stride over rows).  Each row is
+// staged in shared memory by one bulk copy (TMA engine, completion on an
+// mbarrier), double-buffered so the next row streams in while the current one
+// is reduced (row amax) and quantized from shared memory.
+constexpr uint64_t kRowWaitNs = 1000000000ull;
+constexpr uint32_t kBulkPiece = 32768;
+
+template <typename T>
+__device__ __forceinline__ void row_issue(T* dst, const T* src, uint32_t bytes, uint64_t* bar) {
+    sm100::mbar_arrive_expect_tx(bar, bytes);
+    for (uint32_t off = 0; off < bytes; off += kBulkPiece)
+        sm100::bulk_load(reinterpret_cast<uint8_t*>(dst) + off, reinterpret_cast<const uint8_t*>(src) + off,
+                         min(kBulkPiece, bytes - off), bar);
+}
+
+__device__ __forceinline__ void lds8(const uint16_t* p, float v[8]) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+    v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+}
+__device__ __forceinline__ void lds8(const float* p, float v[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+template <typename T>
 __global__ void __launch_bounds__(kThreads) nv_rowamax_quant_kernel(const T* __restrict__ x, int64_t rows, int64_t K,
                                                                     uint8_t* __restrict__ packed,
                                                                     uint8_t* __restrict__ scales,
                                                                     float* __restrict__ g_out) {
+    extern __shared__ __align__(128) uint8_t row_smem[];
     __shared__ float red[32];
-    constexpr int VW = Elem<T>::kBytes * 8 / 16;  // 16-byte words per chunk
+    __shared__ __align__(8) uint64_t bars[2];
     const int64_t cpr = K / 8;
-    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-        const T* xr = x + r * K;
-        uint4 raw[NCH][VW];
+    const uint32_t row_bytes = (uint32_t)(K * sizeof(T));
+    T* const buf0 = reinterpret_cast<T*>(row_smem);
+    T* const buf1 = reinterpret_cast<T*>(row_smem + row_bytes);
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(&bars[0], 1);
+        sm100::mbar_init(&bars[1], 1);
+        sm100::fence_barrier_init();
+    }
+    __syncthreads();
+    int it = 0;
+    int64_t r = blockIdx.x;
+    if (threadIdx.x == 0 && r < rows) row_issue(buf0, x + r * K, row_bytes, &bars[0]);
+    for (; r < rows; r += gridDim.x, ++it) {
+        const int b = it & 1;
+        if (threadIdx.x == 0 && r + gridDim.x < rows)
+            row_issue(b ? buf0 : buf1, x + (r + gridDim.x) * K, row_bytes, &bars[b ^ 1]);
+        // leave together if the copy never lands (every thread must reach the
+        // same barriers)
+        const bool landed = sm100::mbar_wait(&bars[b], (it >> 1) & 1, kRowWaitNs);
+        if (__syncthreads_or(!landed)) break;
+        const T* row = b ? buf1 : buf0;
         float m = 0.0f;
-#pragma unroll
-        for (int i = 0; i < NCH; ++i) {
-            const int64_t c = threadIdx.x + (int64_t)i * kThreads;
-            if (c < cpr) {
-#pragma unroll
-                for (int k = 0; k < VW; ++k) raw[i][k] = __ldcs(reinterpret_cast<const uint4*>(xr + c * 8) + k);
-            } else {
-#pragma unroll
-                for (int k = 0; k < VW; ++k) raw[i][k] = make_uint4(0, 0, 0, 0);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < NCH; ++i) {
+        for (int64_t c = threadIdx.x; c < cpr; c += kThreads) {
             float v[8];
-            if (Elem<T>::kBytes == 2) {
-                v[0] = bf16_lo(raw[i][0].x); v[1] = bf16_hi(raw[i][0].x); v[2] = bf16_lo(raw[i][0].y);
-                v[3] = bf16_hi(raw[i][0].y); v[4] = bf16_lo(raw[i][0].z); v[5] = bf16_hi(raw[i][0].z);
-                v[6] = bf16_lo(raw[i][0].w); v[7] = bf16_hi(raw[i][0].w);
-            } else {
-                const uint4 a = raw[i][0], b = raw[i][VW - 1];
-                v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y); v[2] = __uint_as_float(a.z);
-                v[3] = __uint_as_float(a.w); v[4] = __uint_as_float(b.x); v[5] = __uint_as_float(b.y);
-                v[6] = __uint_as_float(b.z); v[7] = __uint_as_float(b.w);
-            }
+            lds8(row + c * 8, v);
             m = fmaxf(m, amax8(v));
         }
-        const float amax = block_reduce_max(m, red);
-        const float g = __fdiv_rn(amax, kNvGlobalDiv);
+        const float g = __fdiv_rn(block_reduce_max(m, red), kNvGlobalDiv);
         if (threadIdx.x == 0) g_out[r] = g;
-#pragma unroll
-        for (int i = 0; i < NCH; ++i) {
-            const int64_t c = threadIdx.x + (int64_t)i * kThreads;
-            if (i * kThreads >= cpr) break;  // uniform across the CTA
+        // kThreads is even, so the two lanes of a 16-block stay in one warp
+        for (int64_t c0 = 0; c0 < cpr; c0 += kThreads) {
+            const int64_t c = c0 + threadIdx.x;
             float v[8];
-            if (Elem<T>::kBytes == 2) {
-                v[0] = bf16_lo(raw[i][0].x); v[1] = bf16_hi(raw[i][0].x); v[2] = bf16_lo(raw[i][0].y);
-                v[3] = bf16_hi(raw[i][0].y); v[4] = bf16_lo(raw[i][0].z); v[5] = bf16_hi(raw[i][0].z);
-                v[6] = bf16_lo(raw[i][0].w); v[7] = bf16_hi(raw[i][0].w);
-            } else {
-                const uint4 a = raw[i][0], b = raw[i][VW - 1];
-                v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y); v[2] = __uint_as_float(a.z);
-                v[3] = __uint_as_float(a.w); v[4] = __uint_as_float(b.x); v[5] = __uint_as_float(b.y);
-                v[6] = __uint_as_float(b.z); v[7] = __uint_as_float(b.w);
+            if (c < cpr) lds8(row + c * 8, v);
+            else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = 0.0f;
             }
             uint32_t sb;
             const uint32_t pk = nv_quant_chunk(v, g, &sb);
@@ -305,7 +347,11 @@ __global__ void __launch_bounds__(kThreads) nv_rowamax_quant_kernel(const T* __r
                 if ((c & 1) == 0) scales[r * (K / 16) + c / 2] = (uint8_t)sb;
             }
         }
+        __syncthreads();  // the buffer is refilled two rows later
     }
+    // no bulk copy may still be landing in this CTA's shared memory at exit
+    if (threadIdx.x == 0 && r < rows && r + gridDim.x < rows)
+        sm100::mbar_wait(&bars[(it & 1) ^ 1], ((it + 1) >> 1) & 1, kRowWaitNs);
 }
 
 // Row amax for rows too long to keep in registers: pass 1 of the per-row rule.
@@ -559,14 +605,128 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
                 } else {
                     const float s = e4m3_decode(nv_scale_byte(amax_b, g));
                     const float d = __fmul_rn(s, g);
-                    float q[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) q[j] = __fdiv_rn(v[j], d);
-                    const uint32_t pk = e2m1x8_encode_hw(q);
+                    const uint32_t pk = e2m1x8_of_quotient(v, d);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(__fmul_rn(e2m1_decode((pk >> (4 * j)) & 15u), s), g);
                 }
             }
+            if (row_ok && c < cpr && n > 0) {
+                if (VEC && n >= 8) store8(yr + c * 8, out);
+                else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
+            }
+        }
+    }
+}
+
+// Fake-quant of one 8-element chunk in registers (the block's lanes are
+// adjacent; g is the row scale for NVFP4).
+template <int FMT, int L>
+__device__ __forceinline__ void cache_chunk(const float v[8], float g, float out[8]) {
+    const float amax_b = group_max<L>(amax8(v));
+    if (FMT == BSQ_FP8) {
+        const float p = pow2_scale(amax_b, kE4M3Max);
+        const float inv = exp2_int(127 - f32_biased_exp(p));
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            const float2 d = e4m3x2_decode_hw(e4m3x2_encode_hw(v[j] * inv, v[j + 1] * inv));
+            out[j] = d.x * p;
+            out[j + 1] = d.y * p;
+        }
+    } else if (FMT == BSQ_MXFP4) {
+        const float p = pow2_scale(amax_b, kE2M1Max);
+        const float inv = exp2_int(127 - f32_biased_exp(p));
+        float q[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) q[j] = v[j] * inv;
+        const uint32_t pk = e2m1x8_encode_hw(q);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) out[j] = e2m1_decode((pk >> (4 * j)) & 15u) * p;
+    } else {
+        if (g == 0.0f) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) out[j] = 0.0f;
+        } else {
+            const float s = e4m3_decode(nv_scale_byte(amax_b, g));
+            const float d = __fmul_rn(s, g);
+            const uint32_t pk = e2m1x8_of_quotient(v, d);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(__fmul_rn(e2m1_decode((pk >> (4 * j)) & 15u), s), g);
+        }
+    }
+}
+
+// FP8 / MXFP4 fake-quant when every row is a whole number of blocks and
+// 16-byte aligned: the blocks tile the flat tensor, so this is a flat stream
+// with U chunks in flight per lane.
+template <typename T, int FMT, int BLOCK, int U>
+__global__ void __launch_bounds__(kThreads) cache_flat_kernel(const T* __restrict__ x, T* __restrict__ y,
+                                                              int64_t nchunks) {
+    constexpr int L = BLOCK / 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < nchunks; base += U * stride) {
+        float v[U][8];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t c = base + u * stride + lane;
+            if (c < nchunks) load8(x + c * 8, v[u]);
+            else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t c = base + u * stride + lane;
+            float out[8];
+            cache_chunk<FMT, L>(v[u], 0.0f, out);
+            if (c < nchunks) store8(y + c * 8, out);
+        }
+    }
+}
+
+// Row-resident fake-quant: S lanes per row, every lane loads its (at most
+// NCH) chunks of the zero-padded row before any arithmetic; NVFP4 reduces
+// the row amax over the S lanes.  Handles partial groups and ragged C.
+template <typename T, int FMT, int BLOCK, int S, bool VEC, int NCH>
+__global__ void __launch_bounds__(kThreads) cache_row_kernel(const T* __restrict__ x, T* __restrict__ y,
+                                                             int64_t rows, int64_t C) {
+    constexpr int L = BLOCK / 8;
+    constexpr int RPW = 32 / S;
+    const int lane = threadIdx.x & 31;
+    const int sl = lane % S;
+    const int64_t cpr = ((C + BLOCK - 1) / BLOCK) * L;
+    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+    const int64_t wid = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    for (int64_t r0 = wid * RPW; r0 < rows; r0 += warps * RPW) {
+        const int64_t r = r0 + lane / S;
+        const bool row_ok = r < rows;
+        const T* xr = x + (row_ok ? r : 0) * C;
+        T* yr = y + (row_ok ? r : 0) * C;
+        float v[NCH][8];
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            const int64_t c = sl + (int64_t)i * S;
+            const int64_t n = C - c * 8;
+            if (row_ok && c < cpr && n > 0) {
+                if (VEC && n >= 8) load8(xr + c * 8, v[i]);
+                else load_n(xr + c * 8, (int)(n < 8 ? n : 8), v[i]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[i][j] = 0.0f;
+            }
+            m = fmaxf(m, amax8(v[i]));
+        }
+        float g = 0.0f;
+        if (FMT == BSQ_NVFP4) g = __fdiv_rn(group_max<S>(m), kNvGlobalDiv);
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            if (i * S >= cpr) break;  // uniform across the warp
+            const int64_t c = sl + (int64_t)i * S;
+            const int64_t n = C - c * 8;
+            float out[8];
+            cache_chunk<FMT, L>(v[i], g, out);
             if (row_ok && c < cpr && n > 0) {
                 if (VEC && n >= 8) store8(yr + c * 8, out);
                 else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
@@ -624,20 +784,34 @@ static bsq_status check_matrix(const char* fn, const void* x, int64_t rows, int6
         if (_s != BSQ_OK) return _s;       \
     } while (0)
 
+constexpr size_t kRowSmemMax = 100 * 1024;  // two staged rows; longer rows take the two-pass path
+
 template <typename T>
 static bsq_status launch_nv_rowamax(const T* x, int64_t rows, int64_t K, uint8_t* packed, uint8_t* scales,
                                     float* g_out, cudaStream_t st) {
     const int64_t cpr = K / 8;
-    const int nch = (int)((cpr + kThreads - 1) / kThreads);
-    const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * 16);
-#define NV_ROW(N)                                                                                   \
-    if (nch <= N) {                                                                                 \
-        nv_rowamax_quant_kernel<T, N><<<grid, kThreads, 0, st>>>(x, rows, K, packed, scales, g_out); \
-        return check_launch("bsq_quantize_nvfp4");                                                  \
+    const size_t smem = 2 * (size_t)K * sizeof(T);
+    if (smem <= kRowSmemMax) {
+        static std::mutex mu;
+        static bool attr_set[64] = {false};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        {
+            std::lock_guard<std::mutex> lock(mu);
+            if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+                cudaError_t e = cudaFuncSetAttribute(nv_rowamax_quant_kernel<T>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowSmemMax);
+                if (e != cudaSuccess) return fail(BSQ_ERR_CUDA, "bsq_quantize_nvfp4: %s", cudaGetErrorString(e));
+                attr_set[dev] = true;
+            }
+        }
+        const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(8, (200 * 1024) / (smem + 1024)));
+        const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * per_sm);
+        nv_rowamax_quant_kernel<T><<<grid, kThreads, smem, st>>>(x, rows, K, packed, scales, g_out);
+        return check_launch("bsq_quantize_nvfp4");
     }
-    NV_ROW(1) NV_ROW(2) NV_ROW(4) NV_ROW(8) NV_ROW(12) NV_ROW(16)
-#undef NV_ROW
     // long rows: amax pass, then the flat pass with the computed row scales
+    const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * 8);
     row_amax_kernel<T><<<grid, kThreads, 0, st>>>(x, rows, K, g_out);
     BSQ_TRY(check_launch("bsq_quantize_nvfp4"));
     const int64_t nchunks = rows * cpr;
@@ -896,21 +1070,36 @@ BSQ_API bsq_status bsq_dequantize_fp8(const uint8_t* codes_e4m3, const uint8_t* 
     return check_launch("bsq_dequantize_fp8");
 }
 
-template <typename T, int FMT, int BLOCK, bool VEC>
-static void launch_cache_s(const T* x, T* y, int64_t rows, int64_t C, cudaStream_t st) {
-    const int64_t cpr = ((C + BLOCK - 1) / BLOCK) * (BLOCK / 8);
-    int S = 2;
-    while (S < 32 && S < cpr) S <<= 1;
-    if (S < BLOCK / 8) S = BLOCK / 8;
+template <typename T, int FMT, int BLOCK, bool VEC, int S>
+static void launch_cache_rows(const T* x, T* y, int64_t rows, int64_t C, int nch, cudaStream_t st) {
     const int64_t rpw = 32 / S;
     const int64_t warps = (rows + rpw - 1) / rpw;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sm_count() * 8));
+    if (nch <= 1) cache_row_kernel<T, FMT, BLOCK, S, VEC, 1><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+    else if (nch <= 2) cache_row_kernel<T, FMT, BLOCK, S, VEC, 2><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+    else if (nch <= 3) cache_row_kernel<T, FMT, BLOCK, S, VEC, 3><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+    else if (nch <= 4) cache_row_kernel<T, FMT, BLOCK, S, VEC, 4><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+    else cache_kernel<T, FMT, BLOCK, S, VEC><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+}
+
+template <typename T, int FMT, int BLOCK, bool VEC>
+static void launch_cache_s(const T* x, T* y, int64_t rows, int64_t C, cudaStream_t st) {
+    const int64_t cpr = ((C + BLOCK - 1) / BLOCK) * (BLOCK / 8);
+    if (FMT != BSQ_NVFP4 && VEC && C % BLOCK == 0) {
+        const int64_t nchunks = rows * C / 8;
+        cache_flat_kernel<T, FMT, BLOCK, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(x, y, nchunks);
+        return;
+    }
+    int S = 2;
+    while (S < 32 && S < cpr) S <<= 1;
+    if (S < BLOCK / 8) S = BLOCK / 8;
+    const int nch = (int)((cpr + S - 1) / S);
     switch (S) {
-        case 2: cache_kernel<T, FMT, BLOCK, 2, VEC><<<grid, kThreads, 0, st>>>(x, y, rows, C); break;
-        case 4: cache_kernel<T, FMT, BLOCK, 4, VEC><<<grid, kThreads, 0, st>>>(x, y, rows, C); break;
-        case 8: cache_kernel<T, FMT, BLOCK, 8, VEC><<<grid, kThreads, 0, st>>>(x, y, rows, C); break;
-        case 16: cache_kernel<T, FMT, BLOCK, 16, VEC><<<grid, kThreads, 0, st>>>(x, y, rows, C); break;
-        default: cache_kernel<T, FMT, BLOCK, 32, VEC><<<grid, kThreads, 0, st>>>(x, y, rows, C); break;
+        case 2: launch_cache_rows<T, FMT, BLOCK, VEC, 2>(x, y, rows, C, nch, st); break;
+        case 4: launch_cache_rows<T, FMT, BLOCK, VEC, 4>(x, y, rows, C, nch, st); break;
+        case 8: launch_cache_rows<T, FMT, BLOCK, VEC, 8>(x, y, rows, C, nch, st); break;
+        case 16: launch_cache_rows<T, FMT, BLOCK, VEC, 16>(x, y, rows, C, nch, st); break;
+        default: launch_cache_rows<T, FMT, BLOCK, VEC, 32>(x, y, rows, C, nch, st); break;
     }
 }
 
