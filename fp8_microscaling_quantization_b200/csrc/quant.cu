@@ -268,11 +268,71 @@ __device__ __forceinline__ uint32_t nv_quant_chunk(const float v[8], float g, ui
     return e2m1x8_of_quotient(v, d);
 }
 
+// ---- one lane per 16-element NVFP4 block --------------------------------
+
+constexpr float kInv6 = 0.16666667f;        // RN(1/6)
+constexpr float kTwoM120 = 7.5231638e-37f;  // 2**-120
+
+// RN(1/g) when g is a normal value whose reciprocal is normal too (the fast
+// paths below rely on it), else 0.
+__device__ __forceinline__ float nv_recip_or_zero(float g) {
+    return (g >= 2.3509887e-38f && g <= 4.2535296e37f) ? __frcp_rn(g) : 0.0f;
+}
+
+// Block scale code e4m3(max(RN(RN(a / 6) / g), 2**-9)), bit-exact.  With
+// rg = RN(1/g), t1 = RN(RN(a * RN(1/6)) * rg) is within 6 * 2**-24 * t of the
+// two-division chain (a normal, g and 1/g normal); the brackets
+// t1 * (1 -+ 2**-20), clamped at 2**-9, enclose the chain's value, and the
+// e4m3 rounding (to nearest even, saturating) is monotone, so equal codes for
+// both brackets are the chain's code.  Otherwise the chain is evaluated.
+__device__ __forceinline__ uint32_t nv_scale_code(float a, float g, float rg) {
+    if (rg != 0.0f && (a == 0.0f || a >= kTwoM120)) {
+        const float t1 = __fmul_rn(__fmul_rn(a, kInv6), rg);
+        const float lo = fmaxf(__fmul_rn(t1, 0.99999905f), kE4M3MinSub);  // 1 - 2**-20
+        const float hi = fmaxf(__fmul_rn(t1, 1.00000095f), kE4M3MinSub);  // 1 + 2**-20
+        const uint32_t c2 = e4m3x2_encode_hw(lo, hi);
+        if ((c2 & 0xFFu) == (c2 >> 8)) return c2 & 0xFFu;
+    }
+    return nv_scale_byte(a, g);
+}
+
+// 16 values -> 8 bytes of packed e2m1 codes (low word: elements 0..7) and the
+// block's e4m3 scale, for row scale g (0: zero row) with rg = nv_recip_or_zero(g).
+__device__ __forceinline__ uint2 nv_quant_block(const float v[16], float g, float rg, uint32_t* scale_byte) {
+    if (g == 0.0f) {
+        *scale_byte = 0u;
+        return make_uint2(0u, 0u);
+    }
+    const float amax_b = fmaxf(amax8(v), amax8(v + 8));
+    const uint32_t s = nv_scale_code(amax_b, g, rg);
+    const float d = __fmul_rn(e4m3_decode(s), g);
+    *scale_byte = s;
+    return make_uint2(e2m1x8_of_quotient(v, d), e2m1x8_of_quotient(v + 8, d));
+}
+
+// 16 consecutive elements (32-byte aligned for bf16).  Plain (L1-cached)
+// loads: the second half of every line a warp touches is then an L1 hit.
+__device__ __forceinline__ void load16(const uint16_t* p, float v[16]) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p), b = *reinterpret_cast<const uint4*>(p + 8);
+    v[0] = bf16_lo(a.x); v[1] = bf16_hi(a.x); v[2] = bf16_lo(a.y); v[3] = bf16_hi(a.y);
+    v[4] = bf16_lo(a.z); v[5] = bf16_hi(a.z); v[6] = bf16_lo(a.w); v[7] = bf16_hi(a.w);
+    v[8] = bf16_lo(b.x); v[9] = bf16_hi(b.x); v[10] = bf16_lo(b.y); v[11] = bf16_hi(b.y);
+    v[12] = bf16_lo(b.z); v[13] = bf16_hi(b.z); v[14] = bf16_lo(b.w); v[15] = bf16_hi(b.w);
+}
+__device__ __forceinline__ void load16(const float* p, float v[16]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 a = reinterpret_cast<const float4*>(p)[q];
+        v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+    }
+}
+
 // Per-row amax rule: one CTA per row (grid-stride over rows).  Each row is
 // staged in shared memory by one bulk copy (TMA engine, completion on an
 // mbarrier), double-buffered so the next row streams in while the current one
 // is reduced (row amax) and quantized from shared memory.
 constexpr uint64_t kRowWaitNs = 1000000000ull;
+constexpr int kRowThreads = 512;
 constexpr uint32_t kBulkPiece = 32768;
 
 template <typename T>
@@ -294,7 +354,7 @@ __device__ __forceinline__ void lds8(const float* p, float v[8]) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) nv_rowamax_quant_kernel(const T* __restrict__ x, int64_t rows, int64_t K,
+__global__ void __launch_bounds__(kRowThreads) nv_rowamax_quant_kernel(const T* __restrict__ x, int64_t rows, int64_t K,
                                                                     uint8_t* __restrict__ packed,
                                                                     uint8_t* __restrict__ scales,
                                                                     float* __restrict__ g_out) {
@@ -324,28 +384,23 @@ __global__ void __launch_bounds__(kThreads) nv_rowamax_quant_kernel(const T* __r
         if (__syncthreads_or(!landed)) break;
         const T* row = b ? buf1 : buf0;
         float m = 0.0f;
-        for (int64_t c = threadIdx.x; c < cpr; c += kThreads) {
+        for (int64_t c = threadIdx.x; c < cpr; c += kRowThreads) {
             float v[8];
             lds8(row + c * 8, v);
             m = fmaxf(m, amax8(v));
         }
         const float g = __fdiv_rn(block_reduce_max(m, red), kNvGlobalDiv);
         if (threadIdx.x == 0) g_out[r] = g;
-        // kThreads is even, so the two lanes of a 16-block stay in one warp
-        for (int64_t c0 = 0; c0 < cpr; c0 += kThreads) {
-            const int64_t c = c0 + threadIdx.x;
-            float v[8];
-            if (c < cpr) lds8(row + c * 8, v);
-            else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[j] = 0.0f;
-            }
+        const float rg = nv_recip_or_zero(g);
+        const int64_t bpr = K / 16;
+        for (int64_t blk = threadIdx.x; blk < bpr; blk += kRowThreads) {
+            float v[16];
+            lds8(row + blk * 16, v);
+            lds8(row + blk * 16 + 8, v + 8);
             uint32_t sb;
-            const uint32_t pk = nv_quant_chunk(v, g, &sb);
-            if (c < cpr) {
-                reinterpret_cast<uint32_t*>(packed + r * (K / 2))[c] = pk;
-                if ((c & 1) == 0) scales[r * (K / 16) + c / 2] = (uint8_t)sb;
-            }
+            const uint2 pk = nv_quant_block(v, g, rg, &sb);
+            reinterpret_cast<uint2*>(packed + r * (K / 2))[blk] = pk;
+            scales[r * bpr + blk] = (uint8_t)sb;
         }
         __syncthreads();  // the buffer is refilled two rows later
     }
@@ -397,54 +452,51 @@ __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const T* __restr
     if (threadIdx.x == 0) partial[blockIdx.x] = r;
 }
 
-// Flat NVFP4 quantization with a known row scale: MODE 0 = per-row scales
-// given in g_in (copied to g_out), MODE 1 = tensor scale from the partial
-// maxima (reduced by every CTA; CTA 0 publishes it), MODE 2 = per-row scales
-// computed by row_amax_kernel into g_out.
+// Flat NVFP4 quantization with a known row scale, one lane per 16-element
+// block: MODE 0 = per-row scales given in g_in (copied to g_out), MODE 1 =
+// tensor scale from the partial maxima (reduced by every CTA; CTA 0 publishes
+// it), MODE 2 = per-row scales computed by row_amax_kernel into g_out.
 template <typename T, int MODE, int U>
-__global__ void __launch_bounds__(kThreads) nv_flat_quant_kernel(const T* __restrict__ x, int64_t nchunks, FastDiv cpr,
+__global__ void __launch_bounds__(kThreads) nv_flat_quant_kernel(const T* __restrict__ x, int64_t nblocks, FastDiv bpr,
                                                                  const float* __restrict__ g_in,
                                                                  const float* __restrict__ partial, int npartial,
                                                                  uint8_t* __restrict__ packed,
                                                                  uint8_t* __restrict__ scales,
                                                                  float* __restrict__ g_out) {
     __shared__ float red[32];
-    float g_tensor = 0.0f;
+    float g_tensor = 0.0f, rg_tensor = 0.0f;
     if (MODE == 1) {
         float m = 0.0f;
         for (int i = threadIdx.x; i < npartial; i += kThreads) m = fmaxf(m, partial[i]);
         g_tensor = __fdiv_rn(block_reduce_max(m, red), kNvGlobalDiv);
+        rg_tensor = nv_recip_or_zero(g_tensor);
         if (blockIdx.x == 0 && threadIdx.x == 0) g_out[0] = g_tensor;
     }
-    const int lane = threadIdx.x & 31;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < nchunks; base += U * stride) {
-        float v[U][8];
+    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nblocks; base += U * stride) {
+        float v[U][16];
         float g[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t c = base + u * stride + lane;
+            const int64_t b = base + u * stride;
             g[u] = g_tensor;
-            if (c < nchunks) {
-                load8(x + c * 8, v[u]);
-                if (MODE != 1) g[u] = (MODE == 0 ? g_in : g_out)[fdiv((uint32_t)c, cpr)];
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+            if (b < nblocks) {
+                load16(x + b * 16, v[u]);
+                if (MODE != 1) g[u] = (MODE == 0 ? g_in : g_out)[fdiv((uint32_t)b, bpr)];
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t c = base + u * stride + lane;
+            const int64_t b = base + u * stride;
+            if (b >= nblocks) continue;
             uint32_t sb;
-            const uint32_t pk = nv_quant_chunk(v[u], g[u], &sb);
-            if (c < nchunks) {
-                reinterpret_cast<uint32_t*>(packed)[c] = pk;
-                if ((c & 1) == 0) scales[c / 2] = (uint8_t)sb;
-                if (MODE == 0) {
-                    const uint32_t row = fdiv((uint32_t)c, cpr);
-                    if ((uint32_t)c == row * cpr.d) g_out[row] = g[u];
-                }
+            const float rg = (MODE == 1) ? rg_tensor : nv_recip_or_zero(g[u]);
+            const uint2 pk = nv_quant_block(v[u], g[u], rg, &sb);
+            reinterpret_cast<uint2*>(packed)[b] = pk;
+            scales[b] = (uint8_t)sb;
+            if (MODE == 0) {
+                const uint32_t row = fdiv((uint32_t)b, bpr);
+                if ((uint32_t)b == row * bpr.d) g_out[row] = g[u];
             }
         }
     }
@@ -621,7 +673,7 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
 // Fake-quant of one 8-element chunk in registers (the block's lanes are
 // adjacent; g is the row scale for NVFP4).
 template <int FMT, int L>
-__device__ __forceinline__ void cache_chunk(const float v[8], float g, float out[8]) {
+__device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg, float out[8]) {
     const float amax_b = group_max<L>(amax8(v));
     if (FMT == BSQ_FP8) {
         const float p = pow2_scale(amax_b, kE4M3Max);
@@ -646,7 +698,7 @@ __device__ __forceinline__ void cache_chunk(const float v[8], float g, float out
 #pragma unroll
             for (int j = 0; j < 8; ++j) out[j] = 0.0f;
         } else {
-            const float s = e4m3_decode(nv_scale_byte(amax_b, g));
+            const float s = e4m3_decode(nv_scale_code(amax_b, g, rg));
             const float d = __fmul_rn(s, g);
             const uint32_t pk = e2m1x8_of_quotient(v, d);
 #pragma unroll
@@ -679,7 +731,7 @@ __global__ void __launch_bounds__(kThreads) cache_flat_kernel(const T* __restric
         for (int u = 0; u < U; ++u) {
             const int64_t c = base + u * stride + lane;
             float out[8];
-            cache_chunk<FMT, L>(v[u], 0.0f, out);
+            cache_chunk<FMT, L>(v[u], 0.0f, 0.0f, out);
             if (c < nchunks) store8(y + c * 8, out);
         }
     }
@@ -718,15 +770,18 @@ __global__ void __launch_bounds__(kThreads) cache_row_kernel(const T* __restrict
             }
             m = fmaxf(m, amax8(v[i]));
         }
-        float g = 0.0f;
-        if (FMT == BSQ_NVFP4) g = __fdiv_rn(group_max<S>(m), kNvGlobalDiv);
+        float g = 0.0f, rg = 0.0f;
+        if (FMT == BSQ_NVFP4) {
+            g = __fdiv_rn(group_max<S>(m), kNvGlobalDiv);
+            rg = nv_recip_or_zero(g);
+        }
 #pragma unroll
         for (int i = 0; i < NCH; ++i) {
             if (i * S >= cpr) break;  // uniform across the warp
             const int64_t c = sl + (int64_t)i * S;
             const int64_t n = C - c * 8;
             float out[8];
-            cache_chunk<FMT, L>(v[i], g, out);
+            cache_chunk<FMT, L>(v[i], g, rg, out);
             if (row_ok && c < cpr && n > 0) {
                 if (VEC && n >= 8) store8(yr + c * 8, out);
                 else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
@@ -805,18 +860,20 @@ static bsq_status launch_nv_rowamax(const T* x, int64_t rows, int64_t K, uint8_t
                 attr_set[dev] = true;
             }
         }
-        const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(8, (200 * 1024) / (smem + 1024)));
+        // as many staged rows per SM as its 228 KiB of shared memory holds
+        const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(4, (228 * 1024) / (smem + 2048)));
         const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * per_sm);
-        nv_rowamax_quant_kernel<T><<<grid, kThreads, smem, st>>>(x, rows, K, packed, scales, g_out);
+        nv_rowamax_quant_kernel<T><<<grid, kRowThreads, smem, st>>>(x, rows, K, packed, scales, g_out);
         return check_launch("bsq_quantize_nvfp4");
     }
     // long rows: amax pass, then the flat pass with the computed row scales
     const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * 8);
     row_amax_kernel<T><<<grid, kThreads, 0, st>>>(x, rows, K, g_out);
     BSQ_TRY(check_launch("bsq_quantize_nvfp4"));
-    const int64_t nchunks = rows * cpr;
-    nv_flat_quant_kernel<T, 2, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(
-        x, nchunks, make_fastdiv((uint32_t)cpr), nullptr, nullptr, 0, packed, scales, g_out);
+    (void)cpr;
+    const int64_t nblocks = rows * (K / 16);
+    nv_flat_quant_kernel<T, 2, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+        x, nblocks, make_fastdiv((uint32_t)(K / 16)), nullptr, nullptr, 0, packed, scales, g_out);
     return check_launch("bsq_quantize_nvfp4");
 }
 
@@ -827,17 +884,17 @@ BSQ_API bsq_status bsq_quantize_nvfp4(const void* x, bsq_dtype xt, int64_t rows,
     BSQ_TRY(check_matrix("bsq_quantize_nvfp4", x, rows, K, 16));
     if (rows * K == 0) return BSQ_OK;
     if (!packed || !scales_e4m3 || !row_scale_out) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4: null output");
-    if (!aligned(x, 16) || !aligned(packed, 4)) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4: misaligned pointer");
+    if (!aligned(x, 16) || !aligned(packed, 8)) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4: misaligned pointer");
     cudaStream_t st = (cudaStream_t)stream;
     if (row_scale_in) {
-        const int64_t nchunks = rows * (K / 8);
-        const FastDiv cpr = make_fastdiv((uint32_t)(K / 8));
+        const int64_t nblocks = rows * (K / 16);
+        const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
         if (xt == BSQ_BF16)
-            nv_flat_quant_kernel<uint16_t, 0, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(
-                (const uint16_t*)x, nchunks, cpr, row_scale_in, nullptr, 0, packed, scales_e4m3, row_scale_out);
+            nv_flat_quant_kernel<uint16_t, 0, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+                (const uint16_t*)x, nblocks, bpr, row_scale_in, nullptr, 0, packed, scales_e4m3, row_scale_out);
         else
-            nv_flat_quant_kernel<float, 0, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(
-                (const float*)x, nchunks, cpr, row_scale_in, nullptr, 0, packed, scales_e4m3, row_scale_out);
+            nv_flat_quant_kernel<float, 0, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+                (const float*)x, nblocks, bpr, row_scale_in, nullptr, 0, packed, scales_e4m3, row_scale_out);
         return check_launch("bsq_quantize_nvfp4");
     }
     if (xt == BSQ_BF16) return launch_nv_rowamax((const uint16_t*)x, rows, K, packed, scales_e4m3, row_scale_out, st);
@@ -867,25 +924,25 @@ BSQ_API bsq_status bsq_quantize_nvfp4_tensor(const void* x, bsq_dtype xt, int64_
         return BSQ_OK;
     }
     if (!packed || !scales_e4m3 || !scratch) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor: null pointer");
-    if (!aligned(x, 16) || !aligned(packed, 4) || !aligned(scratch, 16))
+    if (!aligned(x, 16) || !aligned(packed, 8) || !aligned(scratch, 16))
         return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor: misaligned pointer");
     const int P = tensor_partials(rows, K);
     if (scratch_bytes < (size_t)P * sizeof(float))
         return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor: scratch of %zu bytes, need %zu", scratch_bytes,
                     (size_t)P * sizeof(float));
-    const int64_t nchunks = rows * (K / 8);
+    const int64_t nchunks = rows * (K / 8), nblocks = rows * (K / 16);
     float* partial = (float*)scratch;
-    const FastDiv cpr = make_fastdiv((uint32_t)(K / 8));
+    const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
     if (xt == BSQ_BF16) {
         amax_partial_kernel<uint16_t, 4><<<P, kThreads, 0, st>>>((const uint16_t*)x, nchunks, partial);
         BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor"));
-        nv_flat_quant_kernel<uint16_t, 1, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(
-            (const uint16_t*)x, nchunks, cpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+        nv_flat_quant_kernel<uint16_t, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+            (const uint16_t*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
     } else {
         amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
         BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor"));
-        nv_flat_quant_kernel<float, 1, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(
-            (const float*)x, nchunks, cpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+        nv_flat_quant_kernel<float, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+            (const float*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
     }
     return check_launch("bsq_quantize_nvfp4_tensor");
 }
@@ -942,7 +999,7 @@ BSQ_API bsq_status bsq_quantize_nvfp4_tensor_noalloc(const void* x, bsq_dtype xt
         return BSQ_OK;
     }
     if (!packed || !scales_e4m3) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor_noalloc: null pointer");
-    if (!aligned(x, 16) || !aligned(packed, 4))
+    if (!aligned(x, 16) || !aligned(packed, 8))
         return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor_noalloc: misaligned pointer");
     const int P = tensor_partials(rows, K);
     if (P > kNoAllocMaxPartials)
@@ -952,18 +1009,18 @@ BSQ_API bsq_status bsq_quantize_nvfp4_tensor_noalloc(const void* x, bsq_dtype xt
     bsq_status status;
     float* partial = noalloc_partials_ptr(&status);
     if (!partial) return status;
-    const int64_t nchunks = rows * (K / 8);
-    const FastDiv cpr = make_fastdiv((uint32_t)(K / 8));
+    const int64_t nchunks = rows * (K / 8), nblocks = rows * (K / 16);
+    const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
     if (xt == BSQ_BF16) {
         amax_partial_kernel<uint16_t, 4><<<P, kThreads, 0, st>>>((const uint16_t*)x, nchunks, partial);
         BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
-        nv_flat_quant_kernel<uint16_t, 1, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(
-            (const uint16_t*)x, nchunks, cpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+        nv_flat_quant_kernel<uint16_t, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+            (const uint16_t*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
     } else {
         amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
         BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
-        nv_flat_quant_kernel<float, 1, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(
-            (const float*)x, nchunks, cpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+        nv_flat_quant_kernel<float, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+            (const float*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
     }
     return check_launch("bsq_quantize_nvfp4_tensor_noalloc");
 }
