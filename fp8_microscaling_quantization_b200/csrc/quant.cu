@@ -332,7 +332,7 @@ __device__ __forceinline__ void load16(const float* p, float v[16]) {
 // mbarrier), double-buffered so the next row streams in while the current one
 // is reduced (row amax) and quantized from shared memory.
 constexpr uint64_t kRowWaitNs = 1000000000ull;
-constexpr int kRowThreads = 512;
+constexpr int kRowThreads = 256;
 constexpr uint32_t kBulkPiece = 32768;
 
 template <typename T>
@@ -358,55 +358,42 @@ __global__ void __launch_bounds__(kRowThreads) nv_rowamax_quant_kernel(const T* 
                                                                     uint8_t* __restrict__ packed,
                                                                     uint8_t* __restrict__ scales,
                                                                     float* __restrict__ g_out) {
-    extern __shared__ __align__(128) uint8_t row_smem[];
+    // One CTA per row (grid-stride).  Pass 1 streams the row from HBM with
+    // plain cached loads (four blocks in flight per thread) and reduces its
+    // amax; pass 2 reads the same row again -- it is still in L2, only the
+    // rows of the CTAs in flight (a few tens of MB) are live -- and quantizes
+    // one 16-element block per thread.
     __shared__ float red[32];
-    __shared__ __align__(8) uint64_t bars[2];
-    const int64_t cpr = K / 8;
-    const uint32_t row_bytes = (uint32_t)(K * sizeof(T));
-    T* const buf0 = reinterpret_cast<T*>(row_smem);
-    T* const buf1 = reinterpret_cast<T*>(row_smem + row_bytes);
-    if (threadIdx.x == 0) {
-        sm100::mbar_init(&bars[0], 1);
-        sm100::mbar_init(&bars[1], 1);
-        sm100::fence_barrier_init();
-    }
-    __syncthreads();
-    int it = 0;
-    int64_t r = blockIdx.x;
-    if (threadIdx.x == 0 && r < rows) row_issue(buf0, x + r * K, row_bytes, &bars[0]);
-    for (; r < rows; r += gridDim.x, ++it) {
-        const int b = it & 1;
-        if (threadIdx.x == 0 && r + gridDim.x < rows)
-            row_issue(b ? buf0 : buf1, x + (r + gridDim.x) * K, row_bytes, &bars[b ^ 1]);
-        // leave together if the copy never lands (every thread must reach the
-        // same barriers)
-        const bool landed = sm100::mbar_wait(&bars[b], (it >> 1) & 1, kRowWaitNs);
-        if (__syncthreads_or(!landed)) break;
-        const T* row = b ? buf1 : buf0;
+    const int64_t bpr = K / 16;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const T* xr = x + r * K;
         float m = 0.0f;
-        for (int64_t c = threadIdx.x; c < cpr; c += kRowThreads) {
-            float v[8];
-            lds8(row + c * 8, v);
-            m = fmaxf(m, amax8(v));
+        for (int64_t b0 = 0; b0 < bpr; b0 += 4 * kRowThreads) {
+            float v[4][16];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t blk = b0 + u * kRowThreads + threadIdx.x;
+                if (blk < bpr) load16(xr + blk * 16, v[u]);
+                else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[u][j] = 0.0f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) m = fmaxf(m, fmaxf(amax8(v[u]), amax8(v[u] + 8)));
         }
         const float g = __fdiv_rn(block_reduce_max(m, red), kNvGlobalDiv);
         if (threadIdx.x == 0) g_out[r] = g;
         const float rg = nv_recip_or_zero(g);
-        const int64_t bpr = K / 16;
         for (int64_t blk = threadIdx.x; blk < bpr; blk += kRowThreads) {
             float v[16];
-            lds8(row + blk * 16, v);
-            lds8(row + blk * 16 + 8, v + 8);
+            load16(xr + blk * 16, v);
             uint32_t sb;
             const uint2 pk = nv_quant_block(v, g, rg, &sb);
             reinterpret_cast<uint2*>(packed + r * (K / 2))[blk] = pk;
             scales[r * bpr + blk] = (uint8_t)sb;
         }
-        __syncthreads();  // the buffer is refilled two rows later
     }
-    // no bulk copy may still be landing in this CTA's shared memory at exit
-    if (threadIdx.x == 0 && r < rows && r + gridDim.x < rows)
-        sm100::mbar_wait(&bars[(it & 1) ^ 1], ((it + 1) >> 1) & 1, kRowWaitNs);
 }
 
 // Row amax for rows too long to keep in registers: pass 1 of the per-row rule.
@@ -839,31 +826,13 @@ static bsq_status check_matrix(const char* fn, const void* x, int64_t rows, int6
         if (_s != BSQ_OK) return _s;       \
     } while (0)
 
-constexpr size_t kRowSmemMax = 100 * 1024;  // two staged rows; longer rows take the two-pass path
-
 template <typename T>
 static bsq_status launch_nv_rowamax(const T* x, int64_t rows, int64_t K, uint8_t* packed, uint8_t* scales,
                                     float* g_out, cudaStream_t st) {
     const int64_t cpr = K / 8;
-    const size_t smem = 2 * (size_t)K * sizeof(T);
-    if (smem <= kRowSmemMax) {
-        static std::mutex mu;
-        static bool attr_set[64] = {false};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        {
-            std::lock_guard<std::mutex> lock(mu);
-            if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-                cudaError_t e = cudaFuncSetAttribute(nv_rowamax_quant_kernel<T>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRowSmemMax);
-                if (e != cudaSuccess) return fail(BSQ_ERR_CUDA, "bsq_quantize_nvfp4: %s", cudaGetErrorString(e));
-                attr_set[dev] = true;
-            }
-        }
-        // as many staged rows per SM as its 228 KiB of shared memory holds
-        const int per_sm = (int)std::max<size_t>(1, std::min<size_t>(4, (228 * 1024) / (smem + 2048)));
-        const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * per_sm);
-        nv_rowamax_quant_kernel<T><<<grid, kRowThreads, smem, st>>>(x, rows, K, packed, scales, g_out);
+    if (K <= 65536) {
+        const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * (2048 / kRowThreads));
+        nv_rowamax_quant_kernel<T><<<grid, kRowThreads, 0, st>>>(x, rows, K, packed, scales, g_out);
         return check_launch("bsq_quantize_nvfp4");
     }
     // long rows: amax pass, then the flat pass with the computed row scales
