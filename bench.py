@@ -65,7 +65,9 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "quant": ["quant.cu", "formats.cuh", "host_util.h"],
+    "flat": ["flat.cu", "common.cuh", "formats.cuh", "host_util.h"],
+    "nvfp4": ["nvfp4.cu", "common.cuh", "formats.cuh", "host_util.h"],
+    "cache": ["cache.cu", "common.cuh", "formats.cuh", "host_util.h"],
     "gemm": ["grouped_mm.cu", "tcgen05.cuh", "formats.cuh", "host_util.h"],
 }
 
@@ -82,7 +84,7 @@ def kernel_source_hash(family):
     return h.hexdigest()[:16]
 
 
-def traffic_from_profiles(kernel_key, family="quant"):
+def traffic_from_profiles(kernel_key, family="flat"):
     """Per-launch DRAM bytes (read + write) of a kernel from the committed ncu
     summary profiles/dram_traffic.json, or None if it is missing or was taken
     on different kernel sources."""

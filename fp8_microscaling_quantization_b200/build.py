@@ -18,8 +18,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libbsq.so")
-SOURCES = ["quant.cu", "grouped_mm.cu"]
-HEADERS = ["formats.cuh", "host_util.h", "tcgen05.cuh"]
+SOURCES = ["abi.cu", "flat.cu", "nvfp4.cu", "cache.cu", "grouped_mm.cu"]
+HEADERS = ["common.cuh", "formats.cuh", "host_util.h", "tcgen05.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

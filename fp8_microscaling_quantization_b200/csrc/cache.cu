@@ -1,0 +1,311 @@
+// cache.cu -- quantize_cache fake-quant and its straight-through backward.
+//
+// Formulas: deepseek_v41 quantization page quantize_cache /
+// _CacheQuantization.forward / .backward: quantize then dequantize each group
+// of `block` channels in binary32, one final rounding to the input dtype; a
+// final partial group is zero-padded.
+#include <cstdarg>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "tcgen05.cuh"
+
+namespace bsq {
+
+// ------------------------------------------------------- quantize_cache ----
+// S lanes per row (S a power of two, 2 <= S <= 32; 32/S rows per warp); lane
+// i of a row walks the chunks i, i + S, ...  of the zero-padded row, so the
+// L lanes of a block are adjacent.  VEC: rows are 16-byte aligned and C % 8 == 0.
+
+template <typename T, int FMT, int BLOCK, int S, bool VEC>
+__global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x, T* __restrict__ y, int64_t rows,
+                                                         int64_t C) {
+    constexpr int L = BLOCK / 8;
+    constexpr int RPW = 32 / S;  // rows per warp
+    const int lane = threadIdx.x & 31;
+    const int sl = lane % S;
+    const int64_t nb = (C + BLOCK - 1) / BLOCK;
+    const int64_t cpr = nb * L;  // chunks in the padded row
+    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+    const int64_t wid = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    for (int64_t r0 = wid * RPW; r0 < rows; r0 += warps * RPW) {
+        const int64_t r = r0 + lane / S;
+        const bool row_ok = r < rows;
+        const T* xr = x + (row_ok ? r : 0) * C;
+        T* yr = y + (row_ok ? r : 0) * C;
+        float g = 0.0f;
+        if (FMT == BSQ_NVFP4) {
+            float m = 0.0f;
+            for (int64_t c0 = 0; c0 < cpr; c0 += S) {
+                const int64_t c = c0 + sl;
+                float v[8];
+                const int64_t n = C - c * 8;
+                if (row_ok && c < cpr && n > 0) {
+                    if (VEC && n >= 8) load8(xr + c * 8, v);
+                    else load_n(xr + c * 8, (int)(n < 8 ? n : 8), v);
+                    m = fmaxf(m, amax8(v));
+                }
+            }
+            m = group_max<S>(m);
+            g = __fdiv_rn(m, kNvGlobalDiv);
+        }
+        for (int64_t c0 = 0; c0 < cpr; c0 += S) {
+            const int64_t c = c0 + sl;
+            const int64_t n = C - c * 8;
+            float v[8];
+            if (row_ok && c < cpr && n > 0) {
+                if (VEC && n >= 8) load8(xr + c * 8, v);
+                else load_n(xr + c * 8, (int)(n < 8 ? n : 8), v);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+            }
+            const float amax_b = group_max<L>(amax8(v));
+            float out[8];
+            if (FMT == BSQ_FP8) {
+                const float p = pow2_scale(amax_b, kE4M3Max);
+                const float inv = exp2_int(127 - f32_biased_exp(p));
+#pragma unroll
+                for (int j = 0; j < 8; j += 2) {
+                    const float2 d = e4m3x2_decode_hw(e4m3x2_encode_hw(v[j] * inv, v[j + 1] * inv));
+                    out[j] = d.x * p;
+                    out[j + 1] = d.y * p;
+                }
+            } else if (FMT == BSQ_MXFP4) {
+                const float p = pow2_scale(amax_b, kE2M1Max);
+                const float inv = exp2_int(127 - f32_biased_exp(p));
+                float q[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) q[j] = v[j] * inv;
+                const uint32_t pk = e2m1x8_encode_hw(q);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) out[j] = e2m1_decode((pk >> (4 * j)) & 15u) * p;
+            } else {
+                if (g == 0.0f) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) out[j] = 0.0f;
+                } else {
+                    const float s = e4m3_decode(nv_scale_byte(amax_b, g));
+                    const float d = __fmul_rn(s, g);
+                    const uint32_t pk = e2m1x8_of_quotient(v, d);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(__fmul_rn(e2m1_decode((pk >> (4 * j)) & 15u), s), g);
+                }
+            }
+            if (row_ok && c < cpr && n > 0) {
+                if (VEC && n >= 8) store8(yr + c * 8, out);
+                else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
+            }
+        }
+    }
+}
+
+// Fake-quant of one 8-element chunk in registers (the block's lanes are
+// adjacent; g is the row scale for NVFP4).
+template <int FMT, int L>
+__device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg, float out[8]) {
+    const float amax_b = group_max<L>(amax8(v));
+    if (FMT == BSQ_FP8) {
+        const float p = pow2_scale(amax_b, kE4M3Max);
+        const float inv = exp2_int(127 - f32_biased_exp(p));
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            const float2 d = e4m3x2_decode_hw(e4m3x2_encode_hw(v[j] * inv, v[j + 1] * inv));
+            out[j] = d.x * p;
+            out[j + 1] = d.y * p;
+        }
+    } else if (FMT == BSQ_MXFP4) {
+        const float p = pow2_scale(amax_b, kE2M1Max);
+        const float inv = exp2_int(127 - f32_biased_exp(p));
+        float q[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) q[j] = v[j] * inv;
+        const uint32_t pk = e2m1x8_encode_hw(q);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) out[j] = e2m1_decode((pk >> (4 * j)) & 15u) * p;
+    } else {
+        if (g == 0.0f) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) out[j] = 0.0f;
+        } else {
+            const float s = e4m3_decode(nv_scale_code(amax_b, g, rg));
+            const float d = __fmul_rn(s, g);
+            const uint32_t pk = e2m1x8_of_quotient(v, d);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(__fmul_rn(e2m1_decode((pk >> (4 * j)) & 15u), s), g);
+        }
+    }
+}
+
+// FP8 / MXFP4 fake-quant when every row is a whole number of blocks and
+// 16-byte aligned: the blocks tile the flat tensor, so this is a flat stream
+// with U chunks in flight per lane.
+template <typename T, int FMT, int BLOCK, int U>
+__global__ void __launch_bounds__(kThreads) cache_flat_kernel(const T* __restrict__ x, T* __restrict__ y,
+                                                              int64_t nchunks) {
+    constexpr int L = BLOCK / 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < nchunks; base += U * stride) {
+        float v[U][8];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t c = base + u * stride + lane;
+            if (c < nchunks) load8(x + c * 8, v[u]);
+            else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t c = base + u * stride + lane;
+            float out[8];
+            cache_chunk<FMT, L>(v[u], 0.0f, 0.0f, out);
+            if (c < nchunks) store8(y + c * 8, out);
+        }
+    }
+}
+
+// Row-resident fake-quant: S lanes per row, every lane loads its (at most
+// NCH) chunks of the zero-padded row before any arithmetic; NVFP4 reduces
+// the row amax over the S lanes.  Handles partial groups and ragged C.
+template <typename T, int FMT, int BLOCK, int S, bool VEC, int NCH>
+__global__ void __launch_bounds__(kThreads) cache_row_kernel(const T* __restrict__ x, T* __restrict__ y,
+                                                             int64_t rows, int64_t C) {
+    constexpr int L = BLOCK / 8;
+    constexpr int RPW = 32 / S;
+    const int lane = threadIdx.x & 31;
+    const int sl = lane % S;
+    const int64_t cpr = ((C + BLOCK - 1) / BLOCK) * L;
+    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+    const int64_t wid = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    for (int64_t r0 = wid * RPW; r0 < rows; r0 += warps * RPW) {
+        const int64_t r = r0 + lane / S;
+        const bool row_ok = r < rows;
+        const T* xr = x + (row_ok ? r : 0) * C;
+        T* yr = y + (row_ok ? r : 0) * C;
+        float v[NCH][8];
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            const int64_t c = sl + (int64_t)i * S;
+            const int64_t n = C - c * 8;
+            if (row_ok && c < cpr && n > 0) {
+                if (VEC && n >= 8) load8(xr + c * 8, v[i]);
+                else load_n(xr + c * 8, (int)(n < 8 ? n : 8), v[i]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[i][j] = 0.0f;
+            }
+            m = fmaxf(m, amax8(v[i]));
+        }
+        float g = 0.0f, rg = 0.0f;
+        if (FMT == BSQ_NVFP4) {
+            g = __fdiv_rn(group_max<S>(m), kNvGlobalDiv);
+            rg = nv_recip_or_zero(g);
+        }
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            if (i * S >= cpr) break;  // uniform across the warp
+            const int64_t c = sl + (int64_t)i * S;
+            const int64_t n = C - c * 8;
+            float out[8];
+            cache_chunk<FMT, L>(v[i], g, rg, out);
+            if (row_ok && c < cpr && n > 0) {
+                if (VEC && n >= 8) store8(yr + c * 8, out);
+                else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
+            }
+        }
+    }
+}
+
+}  // namespace bsq
+
+using namespace bsq;
+
+template <typename T, int FMT, int BLOCK, bool VEC, int S>
+static void launch_cache_rows(const T* x, T* y, int64_t rows, int64_t C, int nch, cudaStream_t st) {
+    const int64_t rpw = 32 / S;
+    const int64_t warps = (rows + rpw - 1) / rpw;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sm_count() * 8));
+    if (nch <= 1) cache_row_kernel<T, FMT, BLOCK, S, VEC, 1><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+    else if (nch <= 2) cache_row_kernel<T, FMT, BLOCK, S, VEC, 2><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+    else if (nch <= 3) cache_row_kernel<T, FMT, BLOCK, S, VEC, 3><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+    else if (nch <= 4) cache_row_kernel<T, FMT, BLOCK, S, VEC, 4><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+    else cache_kernel<T, FMT, BLOCK, S, VEC><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+}
+
+template <typename T, int FMT, int BLOCK, bool VEC>
+static void launch_cache_s(const T* x, T* y, int64_t rows, int64_t C, cudaStream_t st) {
+    const int64_t cpr = ((C + BLOCK - 1) / BLOCK) * (BLOCK / 8);
+    if (FMT != BSQ_NVFP4 && VEC && C % BLOCK == 0) {
+        const int64_t nchunks = rows * C / 8;
+        cache_flat_kernel<T, FMT, BLOCK, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(x, y, nchunks);
+        return;
+    }
+    int S = 2;
+    while (S < 32 && S < cpr) S <<= 1;
+    if (S < BLOCK / 8) S = BLOCK / 8;
+    const int nch = (int)((cpr + S - 1) / S);
+    switch (S) {
+        case 2: launch_cache_rows<T, FMT, BLOCK, VEC, 2>(x, y, rows, C, nch, st); break;
+        case 4: launch_cache_rows<T, FMT, BLOCK, VEC, 4>(x, y, rows, C, nch, st); break;
+        case 8: launch_cache_rows<T, FMT, BLOCK, VEC, 8>(x, y, rows, C, nch, st); break;
+        case 16: launch_cache_rows<T, FMT, BLOCK, VEC, 16>(x, y, rows, C, nch, st); break;
+        default: launch_cache_rows<T, FMT, BLOCK, VEC, 32>(x, y, rows, C, nch, st); break;
+    }
+}
+
+template <typename T, int FMT>
+static void launch_cache_b(int block, const T* x, T* y, int64_t rows, int64_t C, bool vec, cudaStream_t st) {
+    if (block == 16) {
+        if (vec) launch_cache_s<T, FMT, 16, true>(x, y, rows, C, st);
+        else launch_cache_s<T, FMT, 16, false>(x, y, rows, C, st);
+    } else {
+        if (vec) launch_cache_s<T, FMT, 32, true>(x, y, rows, C, st);
+        else launch_cache_s<T, FMT, 32, false>(x, y, rows, C, st);
+    }
+}
+
+template <typename T>
+static void launch_cache(bsq_format fmt, int block, const T* x, T* y, int64_t rows, int64_t C, bool vec,
+                         cudaStream_t st) {
+    if (fmt == BSQ_FP8) launch_cache_b<T, BSQ_FP8>(block, x, y, rows, C, vec, st);
+    else if (fmt == BSQ_MXFP4) launch_cache_b<T, BSQ_MXFP4>(block, x, y, rows, C, vec, st);
+    else launch_cache_b<T, BSQ_NVFP4>(block, x, y, rows, C, vec, st);
+}
+
+BSQ_API bsq_status bsq_quantize_cache(bsq_format fmt, int block, const void* x, void* y, bsq_dtype t, int64_t rows,
+                                      int64_t C, bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(t));
+    if (fmt != BSQ_FP8 && fmt != BSQ_MXFP4 && fmt != BSQ_NVFP4)
+        return fail(BSQ_ERR_UNSUPPORTED, "bsq_quantize_cache: format %d not supported", (int)fmt);
+    if (block != 16 && block != 32) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_cache: block must be 16 or 32");
+    if (rows < 0 || C < 0) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_cache: negative size");
+    if (rows * C == 0) return BSQ_OK;
+    if (!x || !y) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_cache: null pointer");
+    const size_t es = (t == BSQ_BF16) ? 2 : 4;
+    const char* xb = (const char*)x;
+    const char* yb = (const char*)y;
+    const size_t bytes = (size_t)(rows * C) * es;
+    if (xb < yb + bytes && yb < xb + bytes) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_cache: x and y overlap");
+    const bool vec = aligned(x, 16) && aligned(y, 16) && ((C * (int64_t)es) % 16 == 0) && (C % 8 == 0);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (t == BSQ_BF16) launch_cache(fmt, block, (const uint16_t*)x, (uint16_t*)y, rows, C, vec, st);
+    else launch_cache(fmt, block, (const float*)x, (float*)y, rows, C, vec, st);
+    return check_launch("bsq_quantize_cache");
+}
+
+BSQ_API bsq_status bsq_quantize_cache_backward(const void* grad_out, void* grad_in, bsq_dtype t, int64_t n_elems,
+                                               bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(t));
+    if (n_elems < 0) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_cache_backward: negative size");
+    if (n_elems == 0 || grad_in == grad_out) return BSQ_OK;
+    if (!grad_out || !grad_in) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_cache_backward: null pointer");
+    const size_t bytes = (size_t)n_elems * (t == BSQ_BF16 ? 2 : 4);
+    cudaError_t e = cudaMemcpyAsync(grad_in, grad_out, bytes, cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(BSQ_ERR_CUDA, "bsq_quantize_cache_backward: %s", cudaGetErrorString(e));
+    return BSQ_OK;
+}

@@ -1,0 +1,262 @@
+// common.cuh -- device and host helpers shared by the quantize / dequantize
+// / cache kernels of libbsq: element loads and stores, block reductions, the
+// block-scale rules and the bit-exact NVFP4 code computations.
+#pragma once
+
+#include <algorithm>
+#include <cstdint>
+
+#include "formats.cuh"
+#include "host_util.h"
+
+namespace bsq {
+
+static inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// ---------------------------------------------------------- device helpers --
+
+constexpr int kThreads = 256;
+constexpr float kE2M1Max = 6.0f;       // nvfp4 page E2M1_MAX
+constexpr float kE4M3Max = 448.0f;     // nvfp4 page E4M3_MAX
+constexpr float kE4M3MinSub = 0.001953125f;  // nvfp4 page E4M3_MIN_SUBNORMAL = 2**-9
+constexpr float kF32MinNormal = 1.17549435e-38f;  // 2**-126
+constexpr float kNvGlobalDiv = 2688.0f;  // 6 * 448
+
+template <typename T> struct Elem;
+template <> struct Elem<uint16_t> { static constexpr int kBytes = 2; };
+template <> struct Elem<float> { static constexpr int kBytes = 4; };
+
+// 8 consecutive elements starting at p (16-byte aligned for bf16, 32 for fp32).
+__device__ __forceinline__ void load8(const uint16_t* p, float v[8]) {
+    uint4 w = __ldcs(reinterpret_cast<const uint4*>(p));
+    v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+    v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+}
+__device__ __forceinline__ void load8(const float* p, float v[8]) {
+    float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+    float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+// Up to n (< 8) elements with scalar loads, zero fill (ragged rows).
+__device__ __forceinline__ void load_n(const uint16_t* p, int n, float v[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = (j < n) ? __uint_as_float((uint32_t)p[j] << 16) : 0.0f;
+}
+__device__ __forceinline__ void load_n(const float* p, int n, float v[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = (j < n) ? p[j] : 0.0f;
+}
+
+__device__ __forceinline__ void store8(uint16_t* p, const float v[8]) {
+    uint4 w;
+    w.x = pack_bf16x2(v[0], v[1]); w.y = pack_bf16x2(v[2], v[3]);
+    w.z = pack_bf16x2(v[4], v[5]); w.w = pack_bf16x2(v[6], v[7]);
+    __stcs(reinterpret_cast<uint4*>(p), w);
+}
+__device__ __forceinline__ void store8(float* p, const float v[8]) {
+    __stcs(reinterpret_cast<float4*>(p), make_float4(v[0], v[1], v[2], v[3]));
+    __stcs(reinterpret_cast<float4*>(p) + 1, make_float4(v[4], v[5], v[6], v[7]));
+}
+__device__ __forceinline__ void store_n(uint16_t* p, int n, const float v[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (j < n) {
+            __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+            p[j] = *reinterpret_cast<uint16_t*>(&h);
+        }
+}
+__device__ __forceinline__ void store_n(float* p, int n, const float v[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (j < n) p[j] = v[j];
+}
+
+__device__ __forceinline__ float amax8(const float v[8]) {
+    float m = fabsf(v[0]);
+#pragma unroll
+    for (int j = 1; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+    return m;
+}
+
+// Max over the `L` adjacent lanes that share a block (L = 1, 2, 4, ...).
+template <int L>
+__device__ __forceinline__ float group_max(float m) {
+#pragma unroll
+    for (int o = 1; o < L; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    return m;
+}
+
+__device__ __forceinline__ float block_reduce_max(float m, float* smem /* >= 32 floats */) {
+    m = group_max<32>(m);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();  // smem may still be read from a previous use
+    if (lane == 0) smem[warp] = m;
+    __syncthreads();
+    float r = 0.0f;
+    const int nw = (blockDim.x + 31) >> 5;
+    for (int w = 0; w < nw; ++w) r = fmaxf(r, smem[w]);
+    return r;
+}
+
+// MXFP4 block exponent: floor(log2(amax)) - 2, zero block -> -127, clamped.
+__device__ __forceinline__ int mx_exponent(float amax_b) {
+    int e = (amax_b == 0.0f) ? -127 : floor_log2_exact(amax_b) - 2;
+    return max(-127, min(127, e));
+}
+
+// Power-of-two block scale pow2ceil(max(amax / fmt_max, 2**-126)).
+__device__ __forceinline__ float pow2_scale(float amax_b, float fmt_max) {
+    float a = __fdiv_rn(amax_b, fmt_max);
+    if (a < kF32MinNormal) a = kF32MinNormal;
+    return pow2_ceil_normal(a);
+}
+
+// NVFP4 block scale byte: e4m3(max((amax_b / 6) / g, 2**-9)).
+__device__ __forceinline__ uint32_t nv_scale_byte(float amax_b, float g) {
+    float t = __fdiv_rn(__fdiv_rn(amax_b, kE2M1Max), g);
+    t = fmaxf(t, kE4M3MinSub);
+    return e4m3_encode_sw(t);
+}
+
+// e2m1 byte -> (value of low nibble, value of high nibble), built per CTA.
+__device__ __forceinline__ void build_e2m1_lut(float2* lut) {
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) lut[b] = make_float2(e2m1_decode(b & 15), e2m1_decode(b >> 4));
+    __syncthreads();
+}
+
+// ----------------------------------------------------------------- NVFP4 ----
+
+// Quantize one 8-element chunk whose block partner is lane ^ 1, given the
+// row scale g (g == 0: zero row).  Returns the packed 4 bytes; *scale_byte
+// receives the block's e4m3 scale.
+// e2m1 codes of RN(v[j] / d) for 8 values, bit-exact, mostly without a
+// division.  With r = RN(1/d), q = RN(v * r) lies within 1.5 * 2**-23 * |q| of
+// RN(v / d) (two roundings of 2**-24 each, d and r normal).  The e2m1 rounding
+// is monotone in |q|, so if the two brackets q * (1 - 2**-21) and
+// q * (1 + 2**-21), which enclose RN(v / d), round to the same codes, those
+// are the codes of RN(v / d); only when a bracket straddles a rounding
+// boundary (rare) or d is out of range is the quotient computed by IEEE
+// division.
+__device__ __forceinline__ uint32_t e2m1x8_of_quotient(const float v[8], float d) {
+    if (d >= 2.3509887e-38f /* 2**-125 */ && d <= 4.2535296e37f /* 2**125 */) {
+        const float r = __frcp_rn(d);
+        float lo[8], hi[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float q = __fmul_rn(v[j], r);
+            lo[j] = __fmul_rn(q, 0.99999952f);  // 1 - 2**-21
+            hi[j] = __fmul_rn(q, 1.00000048f);  // 1 + 2**-21
+        }
+        const uint32_t clo = e2m1x8_encode_hw(lo), chi = e2m1x8_encode_hw(hi);
+        if (clo == chi) return clo;
+    }
+    float q[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) q[j] = __fdiv_rn(v[j], d);
+    return e2m1x8_encode_hw(q);
+}
+
+// Quantize one 8-element chunk whose block partner is lane ^ 1, given the
+// row scale g (g == 0: zero row).  Returns the packed 4 bytes; *scale_byte
+// receives the block's e4m3 scale.
+__device__ __forceinline__ uint32_t nv_quant_chunk(const float v[8], float g, uint32_t* scale_byte) {
+    const float amax_b = group_max<2>(amax8(v));
+    if (g == 0.0f) {
+        *scale_byte = 0u;
+        return 0u;
+    }
+    const uint32_t s = nv_scale_byte(amax_b, g);
+    const float d = __fmul_rn(e4m3_decode(s), g);
+    *scale_byte = s;
+    return e2m1x8_of_quotient(v, d);
+}
+
+// ---- one lane per 16-element NVFP4 block --------------------------------
+
+constexpr float kInv6 = 0.16666667f;        // RN(1/6)
+constexpr float kTwoM120 = 7.5231638e-37f;  // 2**-120
+
+// RN(1/g) when g is a normal value whose reciprocal is normal too (the fast
+// paths below rely on it), else 0.
+__device__ __forceinline__ float nv_recip_or_zero(float g) {
+    return (g >= 2.3509887e-38f && g <= 4.2535296e37f) ? __frcp_rn(g) : 0.0f;
+}
+
+// Block scale code e4m3(max(RN(RN(a / 6) / g), 2**-9)), bit-exact.  With
+// rg = RN(1/g), t1 = RN(RN(a * RN(1/6)) * rg) is within 6 * 2**-24 * t of the
+// two-division chain (a normal, g and 1/g normal); the brackets
+// t1 * (1 -+ 2**-20), clamped at 2**-9, enclose the chain's value, and the
+// e4m3 rounding (to nearest even, saturating) is monotone, so equal codes for
+// both brackets are the chain's code.  Otherwise the chain is evaluated.
+__device__ __forceinline__ uint32_t nv_scale_code(float a, float g, float rg) {
+    if (rg != 0.0f && (a == 0.0f || a >= kTwoM120)) {
+        const float t1 = __fmul_rn(__fmul_rn(a, kInv6), rg);
+        const float lo = fmaxf(__fmul_rn(t1, 0.99999905f), kE4M3MinSub);  // 1 - 2**-20
+        const float hi = fmaxf(__fmul_rn(t1, 1.00000095f), kE4M3MinSub);  // 1 + 2**-20
+        const uint32_t c2 = e4m3x2_encode_hw(lo, hi);
+        if ((c2 & 0xFFu) == (c2 >> 8)) return c2 & 0xFFu;
+    }
+    return nv_scale_byte(a, g);
+}
+
+// 16 values -> 8 bytes of packed e2m1 codes (low word: elements 0..7) and the
+// block's e4m3 scale, for row scale g (0: zero row) with rg = nv_recip_or_zero(g).
+__device__ __forceinline__ uint2 nv_quant_block(const float v[16], float g, float rg, uint32_t* scale_byte) {
+    if (g == 0.0f) {
+        *scale_byte = 0u;
+        return make_uint2(0u, 0u);
+    }
+    const float amax_b = fmaxf(amax8(v), amax8(v + 8));
+    const uint32_t s = nv_scale_code(amax_b, g, rg);
+    const float d = __fmul_rn(e4m3_decode(s), g);
+    *scale_byte = s;
+    return make_uint2(e2m1x8_of_quotient(v, d), e2m1x8_of_quotient(v + 8, d));
+}
+
+// 16 consecutive elements (32-byte aligned for bf16).  Plain (L1-cached)
+// loads: the second half of every line a warp touches is then an L1 hit.
+__device__ __forceinline__ void load16(const uint16_t* p, float v[16]) {
+    const uint4 a = *reinterpret_cast<const uint4*>(p), b = *reinterpret_cast<const uint4*>(p + 8);
+    v[0] = bf16_lo(a.x); v[1] = bf16_hi(a.x); v[2] = bf16_lo(a.y); v[3] = bf16_hi(a.y);
+    v[4] = bf16_lo(a.z); v[5] = bf16_hi(a.z); v[6] = bf16_lo(a.w); v[7] = bf16_hi(a.w);
+    v[8] = bf16_lo(b.x); v[9] = bf16_hi(b.x); v[10] = bf16_lo(b.y); v[11] = bf16_hi(b.y);
+    v[12] = bf16_lo(b.z); v[13] = bf16_hi(b.z); v[14] = bf16_lo(b.w); v[15] = bf16_hi(b.w);
+}
+__device__ __forceinline__ void load16(const float* p, float v[16]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const float4 a = reinterpret_cast<const float4*>(p)[q];
+        v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
+    }
+}
+
+// Grid of a multiple of the SM count: enough CTAs for `items` at
+// `per_thread` items per thread, capped at 8 CTAs per SM (grid-stride loops).
+static inline int grid_for(int64_t items, int per_thread) {
+    const int64_t need = (items + (int64_t)kThreads * per_thread - 1) / ((int64_t)kThreads * per_thread);
+    const int64_t cap = (int64_t)sm_count() * 8;
+    return (int)std::max<int64_t>(1, std::min(need, cap));
+}
+
+static inline bsq_status check_dtype(bsq_dtype t) {
+    if (t != BSQ_BF16 && t != BSQ_FP32) return fail(BSQ_ERR_UNSUPPORTED, "dtype %d not supported", (int)t);
+    return BSQ_OK;
+}
+
+static inline bsq_status check_matrix(const char* fn, const void* x, int64_t rows, int64_t K, int block) {
+    if (rows < 0 || K < 0) return fail(BSQ_ERR_INVALID_ARG, "%s: negative size (rows=%lld, K=%lld)", fn, (long long)rows, (long long)K);
+    if (K % block != 0)
+        return fail(BSQ_ERR_INVALID_ARG, "%s: K=%lld is not a whole number of %d-column blocks", fn, (long long)K, block);
+    if (rows * K > 0 && x == nullptr) return fail(BSQ_ERR_INVALID_ARG, "%s: null pointer", fn);
+    if (rows * K / 8 >= (int64_t(1) << 32)) return fail(BSQ_ERR_UNSUPPORTED, "%s: tensor too large", fn);
+    return BSQ_OK;
+}
+
+#define BSQ_TRY(expr)                      \
+    do {                                   \
+        bsq_status _s = (expr);            \
+        if (_s != BSQ_OK) return _s;       \
+    } while (0)
+
+
+}  // namespace bsq

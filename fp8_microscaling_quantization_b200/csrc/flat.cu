@@ -1,0 +1,259 @@
+// flat.cu -- MXFP4 and FP8 (power-of-two) quantize, and dequantize for all formats.
+//
+// Work unit: a "chunk" of 8 consecutive elements (one 16-byte bf16 vector).
+// A 16- or 32-column block spans 2 or 4 adjacent lanes of a warp, so the
+// block amax is one or two warp shuffles.  Loads are 128-bit streaming
+// loads; every warp store instruction writes one contiguous span.  Grids are
+// multiples of the SM count with several chunks in flight per thread.
+//
+// Formulas: mxfp4 page quantize_mxfp4 / dequantize_mxfp4; nvfp4 page
+// dequantize_nvfp4; deepseek_v41 quantization page quantize_cache ("fp8"),
+// _power_of_two_ceiling.
+#include <cstdarg>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "tcgen05.cuh"
+
+namespace bsq {
+
+// ----------------------------------------------------------- MXFP4 / FP8 ----
+// Flat block quantization (blocks never cross rows because K % block == 0).
+
+template <typename T, int FMT /*0 = fp8, 1 = mxfp4*/, int BLOCK, int U>
+__global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restrict__ x, int64_t nchunks,
+                                                              uint8_t* __restrict__ codes,
+                                                              uint8_t* __restrict__ scales) {
+    constexpr int L = BLOCK / 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < nchunks; base += U * stride) {
+        float v[U][8];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t c = base + u * stride + lane;
+            if (c < nchunks) load8(x + c * 8, v[u]);
+            else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t c = base + u * stride + lane;
+            const float amax_b = group_max<L>(amax8(v[u]));
+            if (FMT == 1) {
+                const int e = mx_exponent(amax_b);
+                const float inv = exp2_int(-e);  // x * 2**-e == x / 2**e exactly
+                float q[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) q[j] = v[u][j] * inv;
+                const uint32_t packed = e2m1x8_encode_hw(q);
+                if (c < nchunks) {
+                    reinterpret_cast<uint32_t*>(codes)[c] = packed;
+                    if ((lane % L) == 0) scales[c / L] = (uint8_t)(e + 127);
+                }
+            } else {
+                const float p = pow2_scale(amax_b, kE4M3Max);
+                const float inv = exp2_int(127 - f32_biased_exp(p));  // 1 / p, exact
+                uint2 w;
+                w.x = e4m3x2_encode_hw(v[u][0] * inv, v[u][1] * inv) |
+                      (e4m3x2_encode_hw(v[u][2] * inv, v[u][3] * inv) << 16);
+                w.y = e4m3x2_encode_hw(v[u][4] * inv, v[u][5] * inv) |
+                      (e4m3x2_encode_hw(v[u][6] * inv, v[u][7] * inv) << 16);
+                if (c < nchunks) {
+                    reinterpret_cast<uint2*>(codes)[c] = w;
+                    if ((lane % L) == 0) scales[c / L] = (uint8_t)f32_biased_exp(p);
+                }
+            }
+        }
+    }
+}
+
+// Dequantize (all formats).  Item = the EPI consecutive output elements of
+// one lane: 8 for bf16 output (one 16-byte store) and 4 for fp32 output (one
+// 16-byte store), so consecutive lanes write consecutive 16-byte pieces and a
+// warp store instruction covers one contiguous 512-byte span.  FP4 codes are
+// decoded through a 256-entry byte -> (low value, high value) table in shared
+// memory; e4m3 codes through the hardware cvt (exact).
+//   FMT_MX : y = e2m1 * 2**(scale - 127)
+//   FMT_NV : y = (e2m1 * e4m3(scale)) * g[row], row = block / bpr
+//   FMT_FP8: y = e4m3 * 2**(scale - 127)
+enum { FMT_FP8 = 0, FMT_MX = 1, FMT_NV = 2 };
+
+template <int FMT, typename TOUT, int BLOCK, int U>
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __restrict__ codes,
+                                                           const uint8_t* __restrict__ scales,
+                                                           const float* __restrict__ g, FastDiv bpr,
+                                                           int64_t nitems, TOUT* __restrict__ y) {
+    constexpr int EPI = (sizeof(TOUT) == 2) ? 8 : 4;         // elements per item
+    constexpr int CB = (FMT == FMT_FP8) ? EPI : EPI / 2;     // code bytes per item
+    __shared__ float2 lut[256];
+    if (FMT != FMT_FP8) build_e2m1_lut(lut);
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nitems; base += U * stride) {
+        uint32_t w0[U], w1[U], sc[U];
+        float gr[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t it = base + u * stride;
+            w0[u] = w1[u] = sc[u] = 0u;
+            gr[u] = 0.0f;
+            if (it < nitems) {
+                if (CB == 2) w0[u] = __ldcs(reinterpret_cast<const unsigned short*>(codes) + it);
+                else if (CB == 4) w0[u] = __ldcs(reinterpret_cast<const unsigned int*>(codes) + it);
+                else {
+                    const uint2 t = __ldcs(reinterpret_cast<const uint2*>(codes) + it);
+                    w0[u] = t.x;
+                    w1[u] = t.y;
+                }
+                const int64_t blk = (it * EPI) / BLOCK;
+                sc[u] = scales[blk];
+                if (FMT == FMT_NV) gr[u] = g[fdiv((uint32_t)blk, bpr)];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t it = base + u * stride;
+            if (it >= nitems) continue;
+            float v[8];
+            if (FMT == FMT_FP8) {
+                const float p = e8m0_decode(sc[u]);
+#pragma unroll
+                for (int i = 0; i < EPI / 2; ++i) {
+                    const uint32_t word = (i < 2) ? w0[u] : w1[u];
+                    const float2 d = e4m3x2_decode_hw((word >> (16 * (i & 1))) & 0xFFFFu);
+                    v[2 * i] = d.x * p;
+                    v[2 * i + 1] = d.y * p;
+                }
+            } else {
+                const float s = (FMT == FMT_MX) ? e8m0_decode(sc[u]) : e4m3_decode(sc[u]);
+#pragma unroll
+                for (int i = 0; i < EPI / 2; ++i) {
+                    const float2 t = lut[(w0[u] >> (8 * i)) & 0xFFu];
+                    if (FMT == FMT_MX) {
+                        v[2 * i] = t.x * s;
+                        v[2 * i + 1] = t.y * s;
+                    } else {
+                        v[2 * i] = __fmul_rn(__fmul_rn(t.x, s), gr[u]);
+                        v[2 * i + 1] = __fmul_rn(__fmul_rn(t.y, s), gr[u]);
+                    }
+                }
+            }
+            TOUT* dst = y + it * EPI;
+            if (sizeof(TOUT) == 2) {
+                store8(reinterpret_cast<uint16_t*>(dst), v);
+            } else {
+                __stcs(reinterpret_cast<float4*>(dst), make_float4(v[0], v[1], v[2], v[3]));
+            }
+        }
+    }
+}
+
+}  // namespace bsq
+
+using namespace bsq;
+
+BSQ_API bsq_status bsq_dequantize_nvfp4(const uint8_t* packed, const uint8_t* scales_e4m3, const float* row_scale,
+                                        int64_t rows, int64_t K, void* y, bsq_dtype yt, bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(yt));
+    BSQ_TRY(check_matrix("bsq_dequantize_nvfp4", packed, rows, K, 16));
+    if (rows * K == 0) return BSQ_OK;
+    if (!scales_e4m3 || !row_scale || !y) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_nvfp4: null pointer");
+    if (!aligned(packed, 4) || !aligned(y, 16)) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_nvfp4: misaligned pointer");
+    const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (yt == BSQ_BF16) {
+        const int64_t nitems = rows * K / 8;
+        dequant_kernel<FMT_NV, uint16_t, 16, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
+            packed, scales_e4m3, row_scale, bpr, nitems, (uint16_t*)y);
+    } else {
+        const int64_t nitems = rows * K / 4;
+        dequant_kernel<FMT_NV, float, 16, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
+            packed, scales_e4m3, row_scale, bpr, nitems, (float*)y);
+    }
+    return check_launch("bsq_dequantize_nvfp4");
+}
+
+BSQ_API bsq_status bsq_quantize_mxfp4(const void* x, bsq_dtype xt, int64_t rows, int64_t K, uint8_t* packed,
+                                      uint8_t* scales_e8m0, bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(xt));
+    BSQ_TRY(check_matrix("bsq_quantize_mxfp4", x, rows, K, 32));
+    if (rows * K == 0) return BSQ_OK;
+    if (!packed || !scales_e8m0) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_mxfp4: null output");
+    if (!aligned(x, 16) || !aligned(packed, 4)) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_mxfp4: misaligned pointer");
+    const int64_t nchunks = rows * K / 8;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (xt == BSQ_BF16)
+        flat_quant_kernel<uint16_t, 1, 32, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>((const uint16_t*)x, nchunks,
+                                                                                         packed, scales_e8m0);
+    else
+        flat_quant_kernel<float, 1, 32, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>((const float*)x, nchunks, packed,
+                                                                                      scales_e8m0);
+    return check_launch("bsq_quantize_mxfp4");
+}
+
+BSQ_API bsq_status bsq_dequantize_mxfp4(const uint8_t* packed, const uint8_t* scales_e8m0, int64_t rows, int64_t K,
+                                        void* y, bsq_dtype yt, bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(yt));
+    BSQ_TRY(check_matrix("bsq_dequantize_mxfp4", packed, rows, K, 32));
+    if (rows * K == 0) return BSQ_OK;
+    if (!scales_e8m0 || !y) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_mxfp4: null pointer");
+    if (!aligned(packed, 4) || !aligned(y, 16)) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_mxfp4: misaligned pointer");
+    cudaStream_t st = (cudaStream_t)stream;
+    const FastDiv none = make_fastdiv(1);
+    if (yt == BSQ_BF16) {
+        const int64_t nitems = rows * K / 8;
+        dequant_kernel<FMT_MX, uint16_t, 32, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
+            packed, scales_e8m0, nullptr, none, nitems, (uint16_t*)y);
+    } else {
+        const int64_t nitems = rows * K / 4;
+        dequant_kernel<FMT_MX, float, 32, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
+            packed, scales_e8m0, nullptr, none, nitems, (float*)y);
+    }
+    return check_launch("bsq_dequantize_mxfp4");
+}
+
+BSQ_API bsq_status bsq_quantize_fp8(const void* x, bsq_dtype xt, int64_t rows, int64_t K, int block,
+                                    uint8_t* codes_e4m3, uint8_t* scales_e8m0, bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(xt));
+    if (block != 16 && block != 32) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_fp8: block must be 16 or 32");
+    BSQ_TRY(check_matrix("bsq_quantize_fp8", x, rows, K, block));
+    if (rows * K == 0) return BSQ_OK;
+    if (!codes_e4m3 || !scales_e8m0) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_fp8: null output");
+    if (!aligned(x, 16) || !aligned(codes_e4m3, 8)) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_fp8: misaligned pointer");
+    const int64_t nchunks = rows * K / 8;
+    const int grid = grid_for(nchunks, 4);
+    cudaStream_t st = (cudaStream_t)stream;
+    if (xt == BSQ_BF16) {
+        if (block == 32) flat_quant_kernel<uint16_t, 0, 32, 4><<<grid, kThreads, 0, st>>>((const uint16_t*)x, nchunks, codes_e4m3, scales_e8m0);
+        else flat_quant_kernel<uint16_t, 0, 16, 4><<<grid, kThreads, 0, st>>>((const uint16_t*)x, nchunks, codes_e4m3, scales_e8m0);
+    } else {
+        if (block == 32) flat_quant_kernel<float, 0, 32, 4><<<grid, kThreads, 0, st>>>((const float*)x, nchunks, codes_e4m3, scales_e8m0);
+        else flat_quant_kernel<float, 0, 16, 4><<<grid, kThreads, 0, st>>>((const float*)x, nchunks, codes_e4m3, scales_e8m0);
+    }
+    return check_launch("bsq_quantize_fp8");
+}
+
+BSQ_API bsq_status bsq_dequantize_fp8(const uint8_t* codes_e4m3, const uint8_t* scales_e8m0, int64_t rows, int64_t K,
+                                      int block, void* y, bsq_dtype yt, bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(yt));
+    if (block != 16 && block != 32) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_fp8: block must be 16 or 32");
+    BSQ_TRY(check_matrix("bsq_dequantize_fp8", codes_e4m3, rows, K, block));
+    if (rows * K == 0) return BSQ_OK;
+    if (!scales_e8m0 || !y) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_fp8: null pointer");
+    if (!aligned(codes_e4m3, 8) || !aligned(y, 16)) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_fp8: misaligned pointer");
+    cudaStream_t st = (cudaStream_t)stream;
+    const FastDiv none = make_fastdiv(1);
+    const int64_t nb = rows * K / 8, nf = rows * K / 4;
+    if (yt == BSQ_BF16) {
+        if (block == 32) dequant_kernel<FMT_FP8, uint16_t, 32, 4><<<grid_for(nb, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nb, (uint16_t*)y);
+        else dequant_kernel<FMT_FP8, uint16_t, 16, 4><<<grid_for(nb, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nb, (uint16_t*)y);
+    } else {
+        if (block == 32) dequant_kernel<FMT_FP8, float, 32, 4><<<grid_for(nf, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nf, (float*)y);
+        else dequant_kernel<FMT_FP8, float, 16, 4><<<grid_for(nf, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nf, (float*)y);
+    }
+    return check_launch("bsq_dequantize_fp8");
+}
+

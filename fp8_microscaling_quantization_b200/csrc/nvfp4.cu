@@ -1,0 +1,327 @@
+// nvfp4.cu -- NVFP4 quantize: per-row scale, given row scales, ModelOpt tensor scale.
+//
+// Formulas: nvfp4 page quantize_nvfp4 / quantize_nvfp4_modelopt (ModelOpt
+// convention global = amax / (6 * 448), block_scale = e4m3(amax_b / 6 /
+// global) floored at 2**-9, code = round_to_e2m1(w / (block_scale *
+// global))).  One lane per 16-element block; the e4m3 scale and the e2m1
+// codes are bit-exact with mostly no division (see common.cuh).
+#include <cstdarg>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "tcgen05.cuh"
+
+namespace bsq {
+
+// One CTA per row for the per-row amax rule.
+constexpr int kRowThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) nv_rowamax_quant_kernel(const T* __restrict__ x, int64_t rows, int64_t K,
+                                                                    uint8_t* __restrict__ packed,
+                                                                    uint8_t* __restrict__ scales,
+                                                                    float* __restrict__ g_out) {
+    // One CTA per row (grid-stride).  Pass 1 streams the row from HBM with
+    // plain cached loads (four blocks in flight per thread) and reduces its
+    // amax; pass 2 reads the same row again -- it is still in L2, only the
+    // rows of the CTAs in flight (a few tens of MB) are live -- and quantizes
+    // one 16-element block per thread.
+    __shared__ float red[32];
+    const int64_t bpr = K / 16;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const T* xr = x + r * K;
+        float m = 0.0f;
+        for (int64_t b0 = 0; b0 < bpr; b0 += 4 * kRowThreads) {
+            float v[4][16];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t blk = b0 + u * kRowThreads + threadIdx.x;
+                if (blk < bpr) load16(xr + blk * 16, v[u]);
+                else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) v[u][j] = 0.0f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) m = fmaxf(m, fmaxf(amax8(v[u]), amax8(v[u] + 8)));
+        }
+        const float g = __fdiv_rn(block_reduce_max(m, red), kNvGlobalDiv);
+        if (threadIdx.x == 0) g_out[r] = g;
+        const float rg = nv_recip_or_zero(g);
+        for (int64_t blk = threadIdx.x; blk < bpr; blk += kRowThreads) {
+            float v[16];
+            load16(xr + blk * 16, v);
+            uint32_t sb;
+            const uint2 pk = nv_quant_block(v, g, rg, &sb);
+            reinterpret_cast<uint2*>(packed + r * (K / 2))[blk] = pk;
+            scales[r * bpr + blk] = (uint8_t)sb;
+        }
+    }
+}
+
+// Row amax for rows too long to keep in registers: pass 1 of the per-row rule.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) row_amax_kernel(const T* __restrict__ x, int64_t rows, int64_t K,
+                                                            float* __restrict__ g_out) {
+    __shared__ float red[32];
+    const int64_t cpr = K / 8;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        float m = 0.0f;
+        for (int64_t c = threadIdx.x; c < cpr; c += kThreads) {
+            float v[8];
+            load8(x + r * K + c * 8, v);
+            m = fmaxf(m, amax8(v));
+        }
+        const float amax = block_reduce_max(m, red);
+        if (threadIdx.x == 0) g_out[r] = __fdiv_rn(amax, kNvGlobalDiv);
+    }
+}
+
+// Tensor amax, pass 1 of the ModelOpt layout: one partial maximum per CTA.
+template <typename T, int U>
+__global__ void __launch_bounds__(kThreads) amax_partial_kernel(const T* __restrict__ x, int64_t nchunks,
+                                                                float* __restrict__ partial) {
+    __shared__ float red[32];
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    float m = 0.0f;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nchunks; base += U * stride) {
+        float v[U][8];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t c = base + u * stride;
+            if (c < nchunks) load8(x + c * 8, v[u]);
+            else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) m = fmaxf(m, amax8(v[u]));
+    }
+    const float r = block_reduce_max(m, red);
+    if (threadIdx.x == 0) partial[blockIdx.x] = r;
+}
+
+// Flat NVFP4 quantization with a known row scale, one lane per 16-element
+// block: MODE 0 = per-row scales given in g_in (copied to g_out), MODE 1 =
+// tensor scale from the partial maxima (reduced by every CTA; CTA 0 publishes
+// it), MODE 2 = per-row scales computed by row_amax_kernel into g_out.
+template <typename T, int MODE, int U>
+__global__ void __launch_bounds__(kThreads) nv_flat_quant_kernel(const T* __restrict__ x, int64_t nblocks, FastDiv bpr,
+                                                                 const float* __restrict__ g_in,
+                                                                 const float* __restrict__ partial, int npartial,
+                                                                 uint8_t* __restrict__ packed,
+                                                                 uint8_t* __restrict__ scales,
+                                                                 float* __restrict__ g_out) {
+    __shared__ float red[32];
+    float g_tensor = 0.0f, rg_tensor = 0.0f;
+    if (MODE == 1) {
+        float m = 0.0f;
+        for (int i = threadIdx.x; i < npartial; i += kThreads) m = fmaxf(m, partial[i]);
+        g_tensor = __fdiv_rn(block_reduce_max(m, red), kNvGlobalDiv);
+        rg_tensor = nv_recip_or_zero(g_tensor);
+        if (blockIdx.x == 0 && threadIdx.x == 0) g_out[0] = g_tensor;
+    }
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nblocks; base += U * stride) {
+        float v[U][16];
+        float g[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t b = base + u * stride;
+            g[u] = g_tensor;
+            if (b < nblocks) {
+                load16(x + b * 16, v[u]);
+                if (MODE != 1) g[u] = (MODE == 0 ? g_in : g_out)[fdiv((uint32_t)b, bpr)];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t b = base + u * stride;
+            if (b >= nblocks) continue;
+            uint32_t sb;
+            const float rg = (MODE == 1) ? rg_tensor : nv_recip_or_zero(g[u]);
+            const uint2 pk = nv_quant_block(v[u], g[u], rg, &sb);
+            reinterpret_cast<uint2*>(packed)[b] = pk;
+            scales[b] = (uint8_t)sb;
+            if (MODE == 0) {
+                const uint32_t row = fdiv((uint32_t)b, bpr);
+                if ((uint32_t)b == row * bpr.d) g_out[row] = g[u];
+            }
+        }
+    }
+}
+
+}  // namespace bsq
+
+using namespace bsq;
+
+template <typename T>
+static bsq_status launch_nv_rowamax(const T* x, int64_t rows, int64_t K, uint8_t* packed, uint8_t* scales,
+                                    float* g_out, cudaStream_t st) {
+    const int64_t cpr = K / 8;
+    if (K <= 65536) {
+        const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * (2048 / kRowThreads));
+        nv_rowamax_quant_kernel<T><<<grid, kRowThreads, 0, st>>>(x, rows, K, packed, scales, g_out);
+        return check_launch("bsq_quantize_nvfp4");
+    }
+    // long rows: amax pass, then the flat pass with the computed row scales
+    const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * 8);
+    row_amax_kernel<T><<<grid, kThreads, 0, st>>>(x, rows, K, g_out);
+    BSQ_TRY(check_launch("bsq_quantize_nvfp4"));
+    (void)cpr;
+    const int64_t nblocks = rows * (K / 16);
+    nv_flat_quant_kernel<T, 2, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+        x, nblocks, make_fastdiv((uint32_t)(K / 16)), nullptr, nullptr, 0, packed, scales, g_out);
+    return check_launch("bsq_quantize_nvfp4");
+}
+
+BSQ_API bsq_status bsq_quantize_nvfp4(const void* x, bsq_dtype xt, int64_t rows, int64_t K,
+                                      const float* row_scale_in, uint8_t* packed, uint8_t* scales_e4m3,
+                                      float* row_scale_out, bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(xt));
+    BSQ_TRY(check_matrix("bsq_quantize_nvfp4", x, rows, K, 16));
+    if (rows * K == 0) return BSQ_OK;
+    if (!packed || !scales_e4m3 || !row_scale_out) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4: null output");
+    if (!aligned(x, 16) || !aligned(packed, 8)) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4: misaligned pointer");
+    cudaStream_t st = (cudaStream_t)stream;
+    if (row_scale_in) {
+        const int64_t nblocks = rows * (K / 16);
+        const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
+        if (xt == BSQ_BF16)
+            nv_flat_quant_kernel<uint16_t, 0, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+                (const uint16_t*)x, nblocks, bpr, row_scale_in, nullptr, 0, packed, scales_e4m3, row_scale_out);
+        else
+            nv_flat_quant_kernel<float, 0, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+                (const float*)x, nblocks, bpr, row_scale_in, nullptr, 0, packed, scales_e4m3, row_scale_out);
+        return check_launch("bsq_quantize_nvfp4");
+    }
+    if (xt == BSQ_BF16) return launch_nv_rowamax((const uint16_t*)x, rows, K, packed, scales_e4m3, row_scale_out, st);
+    return launch_nv_rowamax((const float*)x, rows, K, packed, scales_e4m3, row_scale_out, st);
+}
+
+static int tensor_partials(int64_t rows, int64_t K) {
+    const int64_t nchunks = rows * (K / 8);
+    return grid_for(nchunks, 4);
+}
+
+BSQ_API size_t bsq_nvfp4_tensor_scratch_bytes(int64_t rows, int64_t K) {
+    if (rows <= 0 || K <= 0) return 16;
+    return (size_t)((tensor_partials(rows, K) * sizeof(float) + 15) / 16 * 16);
+}
+
+BSQ_API bsq_status bsq_quantize_nvfp4_tensor(const void* x, bsq_dtype xt, int64_t rows, int64_t K, uint8_t* packed,
+                                             uint8_t* scales_e4m3, float* tensor_scale_out, void* scratch,
+                                             size_t scratch_bytes, bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(xt));
+    BSQ_TRY(check_matrix("bsq_quantize_nvfp4_tensor", x, rows, K, 16));
+    if (!tensor_scale_out) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor: null tensor scale");
+    cudaStream_t st = (cudaStream_t)stream;
+    if (rows * K == 0) {
+        if (cudaMemsetAsync(tensor_scale_out, 0, sizeof(float), st) != cudaSuccess)
+            return check_launch("bsq_quantize_nvfp4_tensor");
+        return BSQ_OK;
+    }
+    if (!packed || !scales_e4m3 || !scratch) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor: null pointer");
+    if (!aligned(x, 16) || !aligned(packed, 8) || !aligned(scratch, 16))
+        return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor: misaligned pointer");
+    const int P = tensor_partials(rows, K);
+    if (scratch_bytes < (size_t)P * sizeof(float))
+        return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor: scratch of %zu bytes, need %zu", scratch_bytes,
+                    (size_t)P * sizeof(float));
+    const int64_t nchunks = rows * (K / 8), nblocks = rows * (K / 16);
+    float* partial = (float*)scratch;
+    const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
+    if (xt == BSQ_BF16) {
+        amax_partial_kernel<uint16_t, 4><<<P, kThreads, 0, st>>>((const uint16_t*)x, nchunks, partial);
+        BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor"));
+        nv_flat_quant_kernel<uint16_t, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+            (const uint16_t*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+    } else {
+        amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
+        BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor"));
+        nv_flat_quant_kernel<float, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+            (const float*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+    }
+    return check_launch("bsq_quantize_nvfp4_tensor");
+}
+
+// ----------------------------------------------- no-allocation variant ----
+// Some callers cannot hand the library a scratch buffer: a serving engine that
+// reserves all device memory up front and forbids allocations afterwards, or a
+// plain C caller with no device allocator of its own.  For them the per-tensor
+// NVFP4 quantization can keep its per-CTA partial maxima in this file-scope
+// device array instead.  Every GPU that loads the library holds these 16 KiB
+// until the process exits.  The partial maxima are fully written by the first
+// pass before the second pass reads them, so nothing needs clearing between
+// calls.
+constexpr int kNoAllocMaxPartials = 4096;
+static __device__ __align__(256) float g_noalloc_partials[kNoAllocMaxPartials];
+
+// Device address of g_noalloc_partials, looked up once per device with that
+// device current (in host code the array's name is only a host-side handle).
+static float* noalloc_partials_ptr(bsq_status* st) {
+    static std::mutex mu;
+    static float* ptrs[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        *st = fail(BSQ_ERR_CUDA, "bsq_quantize_nvfp4_tensor_noalloc: no current device (%s)",
+                   cudaGetErrorString(e));
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (ptrs[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+        if (e != cudaSuccess || p == nullptr) {
+            *st = fail(BSQ_ERR_CUDA, "bsq_quantize_nvfp4_tensor_noalloc: cudaGetSymbolAddress failed (%s)",
+                       cudaGetErrorString(e));
+            return nullptr;
+        }
+        ptrs[dev] = (float*)p;
+    }
+    *st = BSQ_OK;
+    return ptrs[dev];
+}
+
+BSQ_API bsq_status bsq_quantize_nvfp4_tensor_noalloc(const void* x, bsq_dtype xt, int64_t rows, int64_t K,
+                                                     uint8_t* packed, uint8_t* scales_e4m3, float* tensor_scale_out,
+                                                     bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(xt));
+    BSQ_TRY(check_matrix("bsq_quantize_nvfp4_tensor_noalloc", x, rows, K, 16));
+    if (!tensor_scale_out) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor_noalloc: null tensor scale");
+    cudaStream_t st = (cudaStream_t)stream;
+    if (rows * K == 0) {
+        if (cudaMemsetAsync(tensor_scale_out, 0, sizeof(float), st) != cudaSuccess)
+            return check_launch("bsq_quantize_nvfp4_tensor_noalloc");
+        return BSQ_OK;
+    }
+    if (!packed || !scales_e4m3) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor_noalloc: null pointer");
+    if (!aligned(x, 16) || !aligned(packed, 8))
+        return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor_noalloc: misaligned pointer");
+    const int P = tensor_partials(rows, K);
+    if (P > kNoAllocMaxPartials)
+        return fail(BSQ_ERR_UNSUPPORTED,
+                    "bsq_quantize_nvfp4_tensor_noalloc: needs %d partial maxima, the built-in scratch holds %d",
+                    P, kNoAllocMaxPartials);
+    bsq_status status;
+    float* partial = noalloc_partials_ptr(&status);
+    if (!partial) return status;
+    const int64_t nchunks = rows * (K / 8), nblocks = rows * (K / 16);
+    const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
+    if (xt == BSQ_BF16) {
+        amax_partial_kernel<uint16_t, 4><<<P, kThreads, 0, st>>>((const uint16_t*)x, nchunks, partial);
+        BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
+        nv_flat_quant_kernel<uint16_t, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+            (const uint16_t*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+    } else {
+        amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
+        BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
+        nv_flat_quant_kernel<float, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
+            (const float*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+    }
+    return check_launch("bsq_quantize_nvfp4_tensor_noalloc");
+}
+
