@@ -14,15 +14,16 @@
 // against a 256-feature by 128-token tile, and a short expert pads its token
 // count only to a multiple of 16.
 //
-// Persistent, warp-specialised CTA (one per SM, 448 threads):
+// Persistent, warp-specialised CTA (one per SM, 704 threads):
 //   warps 0-3   epilogue: tensor memory -> registers (x row scale for NVFP4
 //               forward) -> bf16 -> global; lane = feature, so each store of
 //               a token's 32 features is one coalesced 64-byte row piece
-//   warps 4-11  A producers: packed weights + scales from global (several
-//               k-steps in flight), e2m1 -> bf16 by byte permutes, times the
-//               block scale (bf16x2 multiply), swizzled 16-byte shared stores
-//   warp 12     B producer: TMA loads of 64-token x 64-k activation boxes
-//   warp 13     tensor-memory allocation and the single MMA-issuing thread
+//   warps 4-19  A producers, one 16-weight unit of the k-step per thread:
+//               packed weights + scales from global (several k-steps in
+//               flight), e2m1 -> bf16 by byte permutes, times the block scale
+//               (bf16x2 multiply), swizzled 16-byte shared stores
+//   warp 20     B producer: TMA loads of 64-token x 64-k activation boxes
+//   warp 21     tensor-memory allocation and the single MMA-issuing thread
 // Tile = 128 features x up to 256 tokens, k-step 64; separate rings of 5
 // dequantized-weight slots (16 KiB) and 4 activation slots (32 KiB);
 // two 256-column fp32 accumulators in tensor memory so the epilogue of one
@@ -42,6 +43,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "formats.cuh"
@@ -53,28 +55,42 @@ using namespace sm100;
 
 namespace gmm {
 
-constexpr int WM = 128;   // features per tile (MMA M)
+constexpr int WM = 128;   // features per CTA (the CTA's share of MMA M)
 constexpr int TN = 256;   // tokens per tile at most (MMA N)
 constexpr int BK = 64;
-constexpr int WSTAGES = 5;  // dequantized-weight ring (16 KiB slots)
-constexpr int XSTAGES = 4;  // activation ring (32 KiB slots)
 constexpr int XBOX = 64;  // token rows per TMA box
-constexpr int kEpiWarps = 4, kDqWarps = 8;
-constexpr int kTmaWarp = kEpiWarps + kDqWarps;  // 12
-constexpr int kMmaWarp = kTmaWarp + 1;          // 13
-constexpr int kThreads = (kMmaWarp + 1) * 32;   // 448
+// Weights each producer thread converts per k-step (a "unit": 16 or 32
+// consecutive packed weights of one row); the producer warp count follows.
+// 16 (16 producer warps) keeps more weight loads in flight and measured
+// faster in both directions than 32 (8 warps).
+#ifndef BSQ_GMM_UNIT
+#define BSQ_GMM_UNIT 16
+#endif
+constexpr int kUE = BSQ_GMM_UNIT;
+constexpr int kEpiWarps = 4, kDqWarps = (128 * 64 / kUE) / 32;
+constexpr int kTmaWarp = kEpiWarps + kDqWarps;  // 20
+constexpr int kMmaWarp = kTmaWarp + 1;          // 21
+constexpr int kThreads = (kMmaWarp + 1) * 32;   // 704
 constexpr uint32_t kWStage = WM * BK * 2;       // 16 KiB dequantized weights
-constexpr uint32_t kXStage = TN * BK * 2;       // 32 KiB activations
 constexpr uint32_t kXBoxBytes = XBOX * BK * 2;  // 8 KiB
 constexpr int kMaxExperts = 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kPrefetch = 4;  // k-steps of packed weights in flight per producer thread
 
-constexpr size_t kBarOffset = (size_t)WSTAGES * kWStage + (size_t)XSTAGES * kXStage;
-constexpr int kNumBars = 2 * WSTAGES + 2 * XSTAGES + 5;  // w_full/empty, x_full/empty, acc_full[2], acc_empty[2], drain
-constexpr size_t kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 + 16 /* tmem slot, flags */ +
-                              4 * (2 * kMaxExperts + 2);
+// Shared-memory plan of a CTA group of CG CTAs (1, or a pair with
+// cta_group::2): a ring of dequantized-weight slots and a ring of activation
+// slots; each CTA of a pair holds half of the tile's tokens.
+template <int CG>
+struct Plan {
+    static constexpr int WSTAGES = (CG == 1) ? 5 : 7;
+    static constexpr int XSTAGES = (CG == 1) ? 4 : 6;
+    static constexpr uint32_t kXStage = (TN / CG) * BK * 2;  // 32 KiB or 16 KiB
+    static constexpr size_t kBarOffset = (size_t)WSTAGES * kWStage + (size_t)XSTAGES * kXStage;
+    static constexpr int kNumBars = 2 * WSTAGES + 2 * XSTAGES + 5;
+    static constexpr size_t kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 +
+                                         16 /* tmem slot, flags */ + 4 * (2 * kMaxExperts + 2);
+};
 
 struct Args {
     const uint8_t* packed;
@@ -109,20 +125,22 @@ struct Shared {
     int* seg;        // [E + 1] seg[e] = first row of expert e, seg[E] = offs[E-1]
 };
 
+template <int CG>
 __device__ __forceinline__ Shared carve(uint8_t* raw) {
+    using P = Plan<CG>;
     Shared s;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     s.w = base;
-    s.x = base + WSTAGES * kWStage;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(base + kBarOffset);
+    s.x = base + P::WSTAGES * kWStage;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(base + P::kBarOffset);
     s.w_full = bars;
-    s.w_empty = bars + WSTAGES;
-    s.x_full = bars + 2 * WSTAGES;
-    s.x_empty = bars + 2 * WSTAGES + XSTAGES;
-    s.acc_full = bars + 2 * WSTAGES + 2 * XSTAGES;
+    s.w_empty = bars + P::WSTAGES;
+    s.x_full = bars + 2 * P::WSTAGES;
+    s.x_empty = bars + 2 * P::WSTAGES + P::XSTAGES;
+    s.acc_full = bars + 2 * P::WSTAGES + 2 * P::XSTAGES;
     s.acc_empty = s.acc_full + 2;
     s.drain = s.acc_empty + 2;
-    s.tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+    s.tmem_slot = reinterpret_cast<uint32_t*>(bars + P::kNumBars);
     s.abort = reinterpret_cast<volatile int*>(s.tmem_slot + 1);
     s.tt_prefix = reinterpret_cast<int*>(s.tmem_slot + 4);
     s.seg = s.tt_prefix + kMaxExperts + 1;
@@ -144,6 +162,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const S
     return true;
 }
 
+// f0 is the first feature of the group's tile (CTA r of a pair owns
+// features f0 + 128 r ...).
+template <int CG>
 __device__ __forceinline__ Tile decode_tile(int t, int f_tiles, int E, const Shared& sh) {
     const int tg = t / f_tiles;
     const int ft = t - tg * f_tiles;
@@ -157,7 +178,7 @@ __device__ __forceinline__ Tile decode_tile(int t, int f_tiles, int E, const Sha
     ti.e = lo;
     ti.tok0 = sh.seg[lo] + (tg - sh.tt_prefix[lo]) * TN;
     ti.ntok = min(TN, sh.seg[lo + 1] - ti.tok0);
-    ti.f0 = ft * WM;
+    ti.f0 = ft * WM * CG;
     return ti;
 }
 
@@ -208,53 +229,57 @@ __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t code, float g) {
     return b | (b << 16);
 }
 
-// One producer thread's share of a k-step: 32 consecutive packed weights.
+// One producer thread's share of a k-step: kUE consecutive packed weights.
 struct Unit {
-    uint4 pk;
-    uint32_t sc;  // MXFP4: one e8m0 byte; NVFP4: two e4m3 bytes (16-column halves)
-    float g;      // NVFP4 backward row scale
+    uint32_t w[kUE / 8];  // packed e2m1 codes, 8 per word
+    uint32_t sc;          // MXFP4: one e8m0 byte; NVFP4: kUE/16 e4m3 bytes (16-column blocks)
+    float g;              // NVFP4 backward row scale
 };
 
-// Forward: unit u = (feature row u/2 of the tile, k half u%2).  Backward:
-// unit u = (contraction row u/4 of the k-step, 32-column segment u%4 of the
-// tile's 128 k columns).
+// Forward: unit u = (feature row u / (BK/kUE) of the tile, k segment
+// u % (BK/kUE)).  Backward: unit u = (contraction row u / (WM/kUE) of the
+// k-step, kUE-column segment u % (WM/kUE) of the tile's 128 k columns).
 template <int FMT, int DIR>
 __device__ __forceinline__ void load_unit(Unit& u, const Args& a, const Tile& ti, int ks, int unit) {
     int64_t row;
-    int kcol;  // first weight column (k) of the unit's 32 elements
+    int kcol;  // first weight column (k) of the unit
     if (DIR == BSQ_FWD) {
-        row = (int64_t)ti.e * a.N + ti.f0 + (unit >> 1);
-        kcol = ks * BK + (unit & 1) * 32;
+        constexpr int upr = BK / kUE;
+        row = (int64_t)ti.e * a.N + ti.f0 + unit / upr;
+        kcol = ks * BK + (unit % upr) * kUE;
     } else {
-        row = (int64_t)ti.e * a.N + ks * BK + (unit >> 2);
-        kcol = ti.f0 + (unit & 3) * 32;
+        constexpr int upr = WM / kUE;
+        row = (int64_t)ti.e * a.N + ks * BK + unit / upr;
+        kcol = ti.f0 + (unit % upr) * kUE;
     }
-    u.pk = __ldg(reinterpret_cast<const uint4*>(a.packed + row * (a.K / 2) + kcol / 2));
+    const uint8_t* src = a.packed + row * (a.K / 2) + kcol / 2;
+    if (kUE == 32) {
+        const uint4 t = __ldg(reinterpret_cast<const uint4*>(src));
+        u.w[0] = t.x; u.w[1] = t.y; u.w[kUE / 8 - 2] = t.z; u.w[kUE / 8 - 1] = t.w;
+    } else {
+        const uint2 t = __ldg(reinterpret_cast<const uint2*>(src));
+        u.w[0] = t.x; u.w[1] = t.y;
+    }
     if (FMT == BSQ_MXFP4) {
         u.sc = __ldg(a.scales + row * (a.K / 32) + kcol / 32);
         u.g = 1.0f;
     } else {
-        u.sc = __ldg(reinterpret_cast<const unsigned short*>(a.scales + row * (a.K / 16) + kcol / 16));
+        const uint8_t* sp = a.scales + row * (a.K / 16) + kcol / 16;
+        u.sc = (kUE == 32) ? (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(sp)) : (uint32_t)__ldg(sp);
         u.g = (DIR == BSQ_BWD) ? __ldg(a.row_scale + row) : 1.0f;
     }
 }
 
-// Decode a unit into 16 words of bf16x2 (four 16-byte chunks), block scale applied.
+// Decode a unit into kUE/2 words of bf16x2 (16-byte chunks of 8), block scale applied.
 template <int FMT, int DIR>
-__device__ __forceinline__ void decode_unit(const Unit& u, uint32_t (&v)[16]) {
-    uint32_t s_lo, s_hi;
-    if (FMT == BSQ_MXFP4) {
-        s_lo = s_hi = scale_bf16x2<FMT, false>(u.sc, 0.0f);
-    } else {
-        s_lo = scale_bf16x2<FMT, DIR == BSQ_BWD>(u.sc & 0xFFu, u.g);
-        s_hi = scale_bf16x2<FMT, DIR == BSQ_BWD>(u.sc >> 8, u.g);
-    }
-    const uint32_t words[4] = {u.pk.x, u.pk.y, u.pk.z, u.pk.w};
+__device__ __forceinline__ void decode_unit(const Unit& u, uint32_t (&v)[kUE / 2]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kUE / 8; ++i) {
+        uint32_t sc;
+        if (FMT == BSQ_MXFP4) sc = scale_bf16x2<FMT, false>(u.sc, 0.0f);
+        else sc = scale_bf16x2<FMT, DIR == BSQ_BWD>((u.sc >> (8 * (i / 2))) & 0xFFu, u.g);
         uint32_t t[4];
-        e2m1x8_to_bf16(words[i], t);
-        const uint32_t sc = (i < 2) ? s_lo : s_hi;
+        e2m1x8_to_bf16(u.w[i], t);
 #pragma unroll
         for (int j = 0; j < 4; ++j) v[4 * i + j] = mul_bf16x2(t[j], sc);
     }
@@ -262,47 +287,61 @@ __device__ __forceinline__ void decode_unit(const Unit& u, uint32_t (&v)[16]) {
 
 // Write the decoded unit to its place in the swizzled operand tile.
 template <int DIR>
-__device__ __forceinline__ void store_unit(const uint32_t (&v)[16], uint32_t w_stage, int unit) {
+__device__ __forceinline__ void store_unit(const uint32_t (&v)[kUE / 2], uint32_t w_stage, int unit) {
     // 128-byte shared row of the unit and its first 16-byte chunk in that row
     uint32_t base;
     int r, c0;
     if (DIR == BSQ_FWD) {
-        r = unit >> 1;  // K-major: one row per feature, 8-row atoms of 1 KiB
-        c0 = (unit & 1) * 4;
+        constexpr int upr = BK / kUE;
+        r = unit / upr;  // K-major: one row per feature, 8-row atoms of 1 KiB
+        c0 = (unit % upr) * (kUE / 8);
         base = w_stage + (r >> 3) * 1024 + (r & 7) * 128;
     } else {
-        r = unit >> 2;  // MN-major: one row per contraction index, 64-feature panels
-        const int seg = unit & 3;
-        c0 = (seg & 1) * 4;
-        base = w_stage + (seg >> 1) * (BK * 128) + (r >> 3) * 1024 + (r & 7) * 128;
+        constexpr int upr = WM / kUE;
+        r = unit / upr;  // MN-major: one row per contraction index, 64-feature panels
+        const int col = (unit % upr) * kUE;
+        c0 = (col % 64) / 8;
+        base = w_stage + (col / 64) * (BK * 128) + (r >> 3) * 1024 + (r & 7) * 128;
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < kUE / 8; ++i)
         sts128(base + (uint32_t)(((c0 + i) ^ (r & 7)) << 4), v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
 
-template <int FMT, int DIR>
+// Arrive on the barrier at `bar`'s offset in the leader CTA of the group
+// (the CTA itself when CG == 1).
+template <int CG>
+__device__ __forceinline__ void arrive_leader(uint64_t* bar) {
+    if (CG == 1) mbar_arrive(bar);
+    else mbar_arrive_cluster(mapa_shared(smem_u32(bar), 0));
+}
+
+template <int FMT, int DIR, int CG>
 __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_constant__ CUtensorMap tmap_x, Args args) {
+    using P = Plan<CG>;
     extern __shared__ uint8_t smem_raw[];
-    const Shared sh = carve(smem_raw);
+    const Shared sh = carve<CG>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = args.E;
-    const int f_tiles = (DIR == BSQ_FWD ? args.N : args.K) / WM;
-    const int k_steps = (DIR == BSQ_FWD ? args.K : args.N) / BK;
     const int out_w = (DIR == BSQ_FWD ? args.N : args.K);
+    const int f_tiles = out_w / (WM * CG);
+    const int k_steps = (DIR == BSQ_FWD ? args.K : args.N) / BK;
+    const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int group = blockIdx.x / CG, ngroups = gridDim.x / CG;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < WSTAGES; ++s) {
-            mbar_init(&sh.w_full[s], kDqWarps);
+        for (int s = 0; s < P::WSTAGES; ++s) {
+            mbar_init(&sh.w_full[s], kDqWarps * CG);
             mbar_init(&sh.w_empty[s], 1);
         }
-        for (int s = 0; s < XSTAGES; ++s) {
+        for (int s = 0; s < P::XSTAGES; ++s) {
             mbar_init(&sh.x_full[s], 1);
             mbar_init(&sh.x_empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sh.acc_full[i], 1);
-            mbar_init(&sh.acc_empty[i], kEpiWarps);
+            mbar_init(&sh.acc_empty[i], kEpiWarps * CG);
         }
         mbar_init(sh.drain, 1);
         fence_barrier_init();
@@ -324,12 +363,18 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
         if (bad && blockIdx.x == 0) atomicOr(args.err, (uint32_t)BSQ_DEVERR_BAD_OFFS);
     }
     if (warp == kMmaWarp) {
-        tmem_alloc(sh.tmem_slot, kTmemCols);
-        tmem_relinquish();
+        if (CG == 1) {
+            tmem_alloc(sh.tmem_slot, kTmemCols);
+            tmem_relinquish();
+        } else {
+            tmem_alloc_pair(sh.tmem_slot, kTmemCols);
+            tmem_relinquish_pair();
+        }
     }
     if (warp == kTmaWarp && lane == 0) tma_prefetch_desc(&tmap_x);
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync();  // the peer's barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem = sh.tmem_slot[0];
     const int bad = sh.tmem_slot[2];
@@ -348,12 +393,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
         }
         const int q = warp;  // tensor-memory lane quadrant of this warp = features 32q..32q+31
         int tile_iter = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tile_iter) {
-            const Tile ti = decode_tile(t, f_tiles, E, sh);
+        for (int t = group; t < num_tiles; t += ngroups, ++tile_iter) {
+            const Tile ti = decode_tile<CG>(t, f_tiles, E, sh);
             const int acc = tile_iter & 1;
             if (!wait_bar(&sh.acc_full[acc], (tile_iter >> 1) & 1, sh, args.err)) break;
             tc_fence_after();
-            const int f = ti.f0 + q * 32 + lane;
+            const int f = ti.f0 + WM * (int)rank + q * 32 + lane;
             float gf = 1.0f;
             if (FMT == BSQ_NVFP4 && DIR == BSQ_FWD) gf = __ldg(args.row_scale + (int64_t)ti.e * args.N + f);
             uint16_t* ocol = args.out + (int64_t)ti.tok0 * out_w + f;
@@ -376,19 +421,25 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.acc_empty[acc]);
+            if (lane == 0) arrive_leader<CG>(&sh.acc_empty[acc]);
         }
     } else if (warp < kTmaWarp) {
         // ------------------------------------------------- A (weight) producers
-        const int dq = threadIdx.x - kEpiWarps * 32;  // 0..255 = unit index
+        const int dq = threadIdx.x - kEpiWarps * 32;  // unit index
         const uint32_t w_base = smem_u32(sh.w);
         int my_tiles = 0;
-        if (num_tiles > (int)blockIdx.x) my_tiles = (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1;
+        if (num_tiles > group) my_tiles = (num_tiles - 1 - group) / ngroups + 1;
         const int items = my_tiles * k_steps;
-        // load cursor, kPrefetch k-steps ahead of the stores
-        int lt = blockIdx.x, lks = 0;
+        // load cursor, kPrefetch k-steps ahead of the stores; this CTA's
+        // features start WM * rank into the group's tile
+        int lt = group, lks = 0;
         Tile lti;
-        if (items > 0) lti = decode_tile(lt, f_tiles, E, sh);
+        auto cursor_tile = [&](int t) {
+            Tile ti = decode_tile<CG>(t, f_tiles, E, sh);
+            ti.f0 += WM * (int)rank;
+            return ti;
+        };
+        if (items > 0) lti = cursor_tile(lt);
         Unit buf[kPrefetch];
 #pragma unroll
         for (int b = 0; b < kPrefetch; ++b) {
@@ -396,8 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                 load_unit<FMT, DIR>(buf[b], args, lti, lks, dq);
                 if (++lks == k_steps) {
                     lks = 0;
-                    lt += gridDim.x;
-                    if (lt < num_tiles) lti = decode_tile(lt, f_tiles, E, sh);
+                    lt += ngroups;
+                    if (lt < num_tiles) lti = cursor_tile(lt);
                 }
             }
         }
@@ -409,24 +460,24 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                 if (i < items && ok) {
                     // decode first (off the critical path), refill the buffer, then
                     // wait for the shared-memory slot and only store + signal
-                    uint32_t v[16];
+                    uint32_t v[kUE / 2];
                     decode_unit<FMT, DIR>(buf[b], v);
                     if (i + kPrefetch < items) {
                         load_unit<FMT, DIR>(buf[b], args, lti, lks, dq);
                         if (++lks == k_steps) {
                             lks = 0;
-                            lt += gridDim.x;
-                            if (lt < num_tiles) lti = decode_tile(lt, f_tiles, E, sh);
+                            lt += ngroups;
+                            if (lt < num_tiles) lti = cursor_tile(lt);
                         }
                     }
-                    const int s = i % WSTAGES;
-                    if (!wait_bar(&sh.w_empty[s], ((i / WSTAGES) & 1) ^ 1, sh, args.err)) {
+                    const int s = i % P::WSTAGES;
+                    if (!wait_bar(&sh.w_empty[s], ((i / P::WSTAGES) & 1) ^ 1, sh, args.err)) {
                         ok = false;
                     } else {
                         store_unit<DIR>(v, w_base + s * kWStage, dq);
                         fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&sh.w_full[s]);
+                        if (lane == 0) arrive_leader<CG>(&sh.w_full[s]);
                     }
                 }
             }
@@ -436,64 +487,86 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
         if (lane == 0) {
             int it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-                const Tile ti = decode_tile(t, f_tiles, E, sh);
-                const int nbox = (ti.ntok + XBOX - 1) / XBOX;
+            for (int t = group; t < num_tiles && ok; t += ngroups) {
+                const Tile ti = decode_tile<CG>(t, f_tiles, E, sh);
+                const int n_mma = (ti.ntok + 15) & ~15;
+                const int half = n_mma / CG;  // this CTA's share of the tokens
+                const int nbox = (half + XBOX - 1) / XBOX;
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
-                    const int s = it % XSTAGES;
-                    if (!wait_bar(&sh.x_empty[s], ((it / XSTAGES) & 1) ^ 1, sh, args.err)) {
+                    const int s = it % P::XSTAGES;
+                    if (!wait_bar(&sh.x_empty[s], ((it / P::XSTAGES) & 1) ^ 1, sh, args.err)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&sh.x_full[s], nbox * kXBoxBytes);
-                    for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(sh.x + s * kXStage + b * kXBoxBytes, &tmap_x, &sh.x_full[s], ks * BK,
-                                    ti.tok0 + b * XBOX);
+                    uint8_t* dst = sh.x + s * P::kXStage;
+                    if (CG == 1) {
+                        mbar_arrive_expect_tx(&sh.x_full[s], nbox * kXBoxBytes);
+                        for (int b = 0; b < nbox; ++b)
+                            tma_load_2d(dst + b * kXBoxBytes, &tmap_x, &sh.x_full[s], ks * BK, ti.tok0 + b * XBOX);
+                    } else {
+                        // both CTAs' boxes complete on the leader's barrier
+                        if (leader) mbar_arrive_expect_tx(&sh.x_full[s], 2 * nbox * kXBoxBytes);
+                        const uint32_t bar = mapa_shared(smem_u32(&sh.x_full[s]), 0);
+                        for (int b = 0; b < nbox; ++b)
+                            tma_load_2d_pair(dst + b * kXBoxBytes, &tmap_x, bar, ks * BK,
+                                             ti.tok0 + (int)rank * half + b * XBOX);
+                    }
                 }
             }
-            if (!ok) {
-                // drain the loads still in flight into this CTA's shared memory
-                for (int j = (it > XSTAGES ? it - XSTAGES : 0); j < it; ++j)
-                    mbar_wait(&sh.x_full[j % XSTAGES], (j / XSTAGES) & 1, kWaitNs);
+            if (!ok && leader) {
+                // drain the loads still in flight (a pair's loads all count on
+                // the leader's barriers)
+                for (int j = (it > P::XSTAGES ? it - P::XSTAGES : 0); j < it; ++j)
+                    mbar_wait(&sh.x_full[j % P::XSTAGES], (j / P::XSTAGES) & 1, kWaitNs);
             }
         }
     } else {
-        // ----------------------------------------------------------- MMA
-        if (lane == 0) {
+        // ------------------------------------------------ MMA (leader only)
+        if (lane == 0 && leader) {
             const uint32_t w_base = smem_u32(sh.w), x_base = smem_u32(sh.x);
             int it = 0, tile_iter = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tile_iter) {
-                const Tile ti = decode_tile(t, f_tiles, E, sh);
+            for (int t = group; t < num_tiles && ok; t += ngroups, ++tile_iter) {
+                const Tile ti = decode_tile<CG>(t, f_tiles, E, sh);
                 const uint32_t n_mma = (uint32_t)((ti.ntok + 15) & ~15);
-                const uint32_t idesc = idesc_bf16_ab(WM, n_mma, DIR == BSQ_BWD ? 1u : 0u, 0u);
+                const uint32_t idesc = idesc_bf16_ab(WM * CG, n_mma, DIR == BSQ_BWD ? 1u : 0u, 0u);
                 const int acc = tile_iter & 1;
                 if (!wait_bar(&sh.acc_empty[acc], ((tile_iter >> 1) & 1) ^ 1, sh, args.err)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * TN);
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
-                    const int sw = it % WSTAGES, sx = it % XSTAGES;
-                    if (!wait_bar(&sh.w_full[sw], (it / WSTAGES) & 1, sh, args.err) ||
-                        !wait_bar(&sh.x_full[sx], (it / XSTAGES) & 1, sh, args.err)) {
+                    const int sw = it % P::WSTAGES, sx = it % P::XSTAGES;
+                    if (!wait_bar(&sh.w_full[sw], (it / P::WSTAGES) & 1, sh, args.err) ||
+                        !wait_bar(&sh.x_full[sx], (it / P::XSTAGES) & 1, sh, args.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t ws = w_base + sw * kWStage, xs = x_base + sx * kXStage;
+                    const uint32_t ws = w_base + sw * kWStage, xs = x_base + sx * P::kXStage;
 #pragma unroll
                     for (int k16 = 0; k16 < BK / 16; ++k16) {
                         const uint64_t ad = (DIR == BSQ_FWD) ? smem_desc(ws + k16 * 32, 16, 1024)
                                                              : smem_desc(ws + k16 * 2048, BK * 128, 1024);
                         const uint64_t bd = smem_desc(xs + k16 * 32, 16, 1024);
-                        mma_bf16_ss(d_tmem, ad, bd, idesc, (ks | k16) != 0 ? 1u : 0u);
+                        if (CG == 1) mma_bf16_ss(d_tmem, ad, bd, idesc, (ks | k16) != 0 ? 1u : 0u);
+                        else mma_bf16_ss_pair(d_tmem, ad, bd, idesc, (ks | k16) != 0 ? 1u : 0u);
                     }
-                    mma_commit(&sh.w_empty[sw]);
-                    mma_commit(&sh.x_empty[sx]);
+                    if (CG == 1) {
+                        mma_commit(&sh.w_empty[sw]);
+                        mma_commit(&sh.x_empty[sx]);
+                    } else {
+                        mma_commit_pair_multicast(&sh.w_empty[sw], 0x3);
+                        mma_commit_pair_multicast(&sh.x_empty[sx], 0x3);
+                    }
                 }
-                if (ok) mma_commit(&sh.acc_full[acc]);
+                if (ok) {
+                    if (CG == 1) mma_commit(&sh.acc_full[acc]);
+                    else mma_commit_pair_multicast(&sh.acc_full[acc], 0x3);
+                }
             }
             // every MMA this thread issued has completed once `drain` fires
-            mma_commit(sh.drain);
+            if (CG == 1) mma_commit(sh.drain);
+            else mma_commit_pair_multicast(sh.drain, 0x1);
             mbar_wait(sh.drain, 0, kWaitNs);
         }
     }
@@ -501,8 +574,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
     __syncwarp();
     tc_fence_before();
     __syncthreads();
+    if (CG == 2) cluster_sync();  // no CTA leaves while its peer may still touch it
     tc_fence_after();
-    if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kMmaWarp) {
+        if (CG == 1) tmem_dealloc(tmem, kTmemCols);
+        else tmem_dealloc_pair(tmem, kTmemCols);
+    }
 }
 
 }  // namespace gmm
@@ -532,23 +609,48 @@ static EncodeTiledFn encode_fn(bsq_status* st) {
     return fn;
 }
 
-template <int FMT, int DIR>
-static bsq_status launch_gmm(const CUtensorMap& tmap, const gmm::Args& a, int grid, cudaStream_t st) {
+template <int FMT, int DIR, int CG>
+static bsq_status launch_gmm(const CUtensorMap& tmap, const gmm::Args& a, int64_t max_groups, cudaStream_t st) {
     static std::mutex mu;
-    static bool attr_set[64] = {false};
+    static int max_active[64] = {0};  // co-resident groups per device (0: not yet queried)
+    auto kern = gmm::grouped_mm_kernel<FMT, DIR, CG>;
+    const size_t smem = gmm::Plan<CG>::kSmemBytes;
     int dev = 0;
     cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.blockDim = dim3(gmm::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    if (CG == 2) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
     {
         std::lock_guard<std::mutex> lock(mu);
-        if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-            cudaError_t e = cudaFuncSetAttribute(gmm::grouped_mm_kernel<FMT, DIR>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gmm::kSmemBytes);
+        if (max_active[dev] == 0) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess)
                 return fail(BSQ_ERR_CUDA, "bsq_grouped_mm_fp4: shared-memory opt-in failed (%s)", cudaGetErrorString(e));
-            attr_set[dev] = true;
+            int n = sm_count() / CG;
+            if (CG == 2) {
+                cfg.gridDim = dim3(2 * n, 1, 1);
+                int clusters = 0;
+                if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0) n = clusters;
+                cudaGetLastError();
+            }
+            max_active[dev] = n;
         }
     }
-    gmm::grouped_mm_kernel<FMT, DIR><<<grid, gmm::kThreads, gmm::kSmemBytes, st>>>(tmap, a);
+    const int groups = (int)std::max<int64_t>(1, std::min<int64_t>(max_groups, max_active[dev]));
+    cfg.gridDim = dim3(groups * CG, 1, 1);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmap, a);
+    if (e != cudaSuccess) return fail(BSQ_ERR_CUDA, "bsq_grouped_mm_fp4: launch failed (%s)", cudaGetErrorString(e));
     return check_launch("bsq_grouped_mm_fp4");
 }
 
@@ -603,13 +705,25 @@ BSQ_API bsq_status bsq_grouped_mm_fp4(bsq_format fmt, bsq_dir dir, const void* a
     args.T = (int)T;
     args.N = (int)N;
     args.K = (int)K;
-    const int64_t f_tiles = out_w / gmm::WM;
-    const int64_t max_tiles = ((T + gmm::TN - 1) / gmm::TN + E) * f_tiles;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(max_tiles, sm_count()));
+    // Single CTAs by default.  The environment variable BSQ_GMM_CTA_PAIR=1
+    // selects CTA pairs (M = 256 features per tile, cta_group::2) where the
+    // output width allows it; both measured within a few per cent of each
+    // other with 16-weight producer units.
+    const char* pair_env = getenv("BSQ_GMM_CTA_PAIR");
+    const int cg = (pair_env && pair_env[0] == '1' && out_w % (2 * gmm::WM) == 0) ? 2 : 1;
+    const int64_t f_tiles = out_w / (gmm::WM * cg);
+    const int64_t max_groups = ((T + gmm::TN - 1) / gmm::TN + E) * f_tiles;
     cudaStream_t s = (cudaStream_t)stream;
+    if (cg == 2) {
+        if (fmt == BSQ_MXFP4)
+            return dir == BSQ_FWD ? launch_gmm<BSQ_MXFP4, BSQ_FWD, 2>(tmap, args, max_groups, s)
+                                  : launch_gmm<BSQ_MXFP4, BSQ_BWD, 2>(tmap, args, max_groups, s);
+        return dir == BSQ_FWD ? launch_gmm<BSQ_NVFP4, BSQ_FWD, 2>(tmap, args, max_groups, s)
+                              : launch_gmm<BSQ_NVFP4, BSQ_BWD, 2>(tmap, args, max_groups, s);
+    }
     if (fmt == BSQ_MXFP4)
-        return dir == BSQ_FWD ? launch_gmm<BSQ_MXFP4, BSQ_FWD>(tmap, args, grid, s)
-                              : launch_gmm<BSQ_MXFP4, BSQ_BWD>(tmap, args, grid, s);
-    return dir == BSQ_FWD ? launch_gmm<BSQ_NVFP4, BSQ_FWD>(tmap, args, grid, s)
-                          : launch_gmm<BSQ_NVFP4, BSQ_BWD>(tmap, args, grid, s);
+        return dir == BSQ_FWD ? launch_gmm<BSQ_MXFP4, BSQ_FWD, 1>(tmap, args, max_groups, s)
+                              : launch_gmm<BSQ_MXFP4, BSQ_BWD, 1>(tmap, args, max_groups, s);
+    return dir == BSQ_FWD ? launch_gmm<BSQ_NVFP4, BSQ_FWD, 1>(tmap, args, max_groups, s)
+                          : launch_gmm<BSQ_NVFP4, BSQ_BWD, 1>(tmap, args, max_groups, s);
 }

@@ -100,6 +100,24 @@ def test_gemm_edge_offsets(B, oracle, fmt):
     full_check(B, oracle, fmt, T=64, K=256, N=256, E=3, seed=15, offs=[0, 0, 0])
 
 
+@pytest.mark.parametrize("fmt", [1, 2])
+def test_gemm_cta_pairs(B, oracle, fmt, monkeypatch):
+    # BSQ_GMM_CTA_PAIR=1 runs 256-feature tiles on CTA pairs (cta_group::2);
+    # an output width of 384 is not a multiple of 256 and falls back to single
+    # CTAs within the same call sequence
+    monkeypatch.setenv("BSQ_GMM_CTA_PAIR", "1")
+    full_check(B, oracle, fmt, T=300, K=256, N=256, E=4, seed=11)
+    full_check(B, oracle, fmt, T=2048, K=1024, N=512, E=8, seed=12)
+    full_check(B, oracle, fmt, T=400, K=256, N=256, E=6, seed=14, offs=[0, 1, 130, 130, 390, 390])
+    full_check(B, oracle, fmt, T=300, K=384, N=384, E=3, seed=17)
+
+
+@pytest.mark.parametrize("fmt", [1, 2])
+def test_gemm_output_width_not_256(B, oracle, fmt):
+    # output width a multiple of 128 but not of 256, K not a multiple of 128
+    full_check(B, oracle, fmt, T=300, K=384, N=384, E=3, seed=17)
+
+
 def test_gemm_bad_offs_reported(B, oracle):
     x, w, go, _ = make_problem(256, 256, 256, 4, 16, offs=[0, 0, 0, 0])
     packed, scales, g = quantize_weights(oracle, oracle.FMT_MXFP4, w)
