@@ -37,6 +37,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "quant/dequant GB/s (% HBM peak); dequant grouped-GEMM TFLOP/s (% bf16 peak)"
 E, N, K = 8, 2048, 7168
+# GPU spin (about 100 us at 1.9 GHz) queued in front of a timed launch
+HOST_COVER_CYCLES = 200_000
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -48,7 +50,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the sub-measurements of the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
-    ap.add_argument("--only", default="", help="comma list of extra sections to run (nvfp4,cache,linear,gemm)")
+    ap.add_argument("--only", default="", help="run only these sub-measurements (comma list of nvfp4,cache,linear,"
+                    "gemm) and print them, without the main step; for profiling")
     ap.add_argument("--gemm-only", default="", help="time only these grouped-GEMM variants (comma list of "
                     "mxfp4_fwd,mxfp4_bwd,nvfp4_fwd,nvfp4_bwd) and print them; for profiling")
     return ap.parse_args()
@@ -84,20 +87,26 @@ def kernel_source_hash(family):
     return h.hexdigest()[:16]
 
 
-def traffic_from_profiles(kernel_key, family="flat"):
-    """Per-launch DRAM bytes (read + write) of a kernel from the committed ncu
-    summary profiles/dram_traffic.json, or None if it is missing or was taken
-    on different kernel sources."""
+def traffic_from_profiles(*kernel_keys):
+    """Per-launch DRAM bytes (read + write, summed over the given kernels) from
+    the committed ncu summary profiles/dram_traffic.json, or None if an entry
+    is missing or was taken on other sources than the kernel family's current
+    ones."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
     except Exception:
         return None
-    ent = d.get("kernels", {}).get(kernel_key)
-    if not ent or ent.get("source_hash") != kernel_source_hash(family):
-        return None
-    return ent.get("bytes_per_launch")
+    total = 0
+    for key in kernel_keys:
+        ent = d.get("kernels", {}).get(key)
+        if not ent or ent.get("family") not in KERNEL_SOURCES:
+            return None
+        if ent.get("source_hash") != kernel_source_hash(ent["family"]):
+            return None
+        total += ent.get("bytes_per_launch", 0)
+    return total
 
 
 # ------------------------------------------------------------------ clocks --
@@ -270,6 +279,14 @@ def main():
                          variants=set(args.gemm_only.split(",")), iters=max(1, args.steps), warm=args.warmup)
         print(json.dumps({"grouped_gemm": res}), flush=True)
         return
+    if args.only:
+        from fp8_microscaling_quantization_b200 import bsq, synth
+        peaks, peak_kind = load_peaks()
+        dev = torch.device("cuda", 0)
+        res = run_extra(torch, bsq, synth, dev, torch.cuda.current_stream(), peaks, peak_kind,
+                        set(filter(None, args.only.split(","))))
+        print(json.dumps({"extra": res}), flush=True)
+        return
     import torch.distributed as dist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -382,8 +399,7 @@ def main():
         except Exception as ex:  # report, never hide
             line["cpu_baseline"] = {"unavailable": f"{type(ex).__name__}: {ex}"}
     if not args.no_extra and world == 1:
-        only = set(filter(None, args.only.split(",")))
-        line["extra"] = run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only)
+        line["extra"] = run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, set())
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -443,13 +459,19 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
         for _ in range(iters):
             if cold:
                 l2_flush(torch, flush)
+            # keep the GPU busy while the host enqueues the start event and the
+            # launch, so the event pair brackets the kernel and not host time
+            torch.cuda._sleep(HOST_COVER_CYCLES)
             t.run("k", fn)
         torch.cuda.synchronize()
         return t.avg_ms("k")
 
-    def rec(ms, nbytes):
-        return {"us": round(ms * 1e3, 2), "bytes": nbytes, "GB/s": round(nbytes / ms / 1e6, 1),
-                "frac_hbm": round(nbytes / ms / 1e6 / hbm, 4)}
+    def rec(ms, nbytes, *traffic_keys):
+        r = {"us": round(ms * 1e3, 2), "bytes": nbytes, "GB/s": round(nbytes / ms / 1e6, 1),
+             "frac_hbm": round(nbytes / ms / 1e6 / hbm, 4)}
+        if traffic_keys:
+            r["traffic"] = traffic_from_profiles(*traffic_keys)
+        return r
 
     want = (lambda s: not only or s in only)
 
@@ -477,7 +499,7 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
             x = synth.cache_acts_torch(*shp, generator=g, device=dev)
             y = torch.empty_like(x)
             nb = 2 * 2 * x.numel()
-            res[name] = rec(timed(lambda: bsq.bsq_quantize_cache(x, fmt, blk, y=y), 30, True), nb)
+            res[name] = rec(timed(lambda: bsq.bsq_quantize_cache(x, fmt, blk, y=y), 30, True), nb, "cache_" + name)
         gsrc = torch.randn((4, 8192, 512), generator=g, device=dev).to(torch.bfloat16)
         gdst = torch.empty_like(gsrc)
         res["ste_backward_aliased"] = {"us": 0.0, "bytes": 0, "note": "identity: no launch"}
@@ -510,12 +532,15 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
         nb_dq = n // 2 + n // 16 + 4 * 7168 + 2 * n
         out["nvfp4_linear_7168x18432"] = {
             "modelopt_tensor_scale": rec(timed(lambda: bsq.bsq_quantize_nvfp4_tensor(
-                x, packed=p, scales=s, tensor_scale=t, scratch=scratch), 10, False), nb_tensor),
+                x, packed=p, scales=s, tensor_scale=t, scratch=scratch), 10, False), nb_tensor,
+                "nvfp4_tensor_amax_pass", "nvfp4_tensor_quant_pass"),
             "per_row_scale": rec(timed(lambda: bsq.bsq_quantize_nvfp4(x, packed=p, scales=s, row_scale_out=r),
-                                       10, False), nb_row),
+                                       10, False), nb_row, "nvfp4_per_row"),
             "gate_up_given_row_scales_14336x18432": rec(timed(lambda: bsq.bsq_quantize_nvfp4(
-                cat, row_scale_in=rc, packed=pc, scales=sc, row_scale_out=rco), 10, False), nb_gu),
-            "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_nvfp4(p, s, r, y=y), 10, False), nb_dq),
+                cat, row_scale_in=rc, packed=pc, scales=sc, row_scale_out=rco), 10, False), nb_gu,
+                "nvfp4_gate_up_given_row_scales"),
+            "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_nvfp4(p, s, r, y=y), 10, False), nb_dq,
+                                   "nvfp4_dequant_bf16"),
             "note": "inputs larger than L2; per-tensor counts two reads of the input"}
         del x, cat, y
 
@@ -564,7 +589,8 @@ def bench_gemm(torch, bsq, synth, dev, stream, peaks, peak_kind, variants=None, 
             ms = t.avg_ms("k")
             tf = flops / (ms * 1e-3) / 1e12
             res[f"{fmt_name}_{dname}"] = {"us": round(ms * 1e3, 1), "TFLOP/s": round(tf, 1),
-                                          "frac_bf16": round(tf / peak, 4)}
+                                          "frac_bf16": round(tf / peak, 4),
+                                          "traffic": traffic_from_profiles(f"gemm_{fmt_name}_{dname}")}
     res["err_word"] = int(err.item())
     res["peak"] = f"{peak} TFLOP/s bf16 dense ({peak_kind}, burst)"
     return res
