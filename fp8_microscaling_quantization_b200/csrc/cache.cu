@@ -229,12 +229,12 @@ template <typename T, int FMT, int BLOCK, bool VEC, int S>
 static void launch_cache_rows(const T* x, T* y, int64_t rows, int64_t C, int nch, cudaStream_t st) {
     const int64_t rpw = 32 / S;
     const int64_t warps = (rows + rpw - 1) / rpw;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((warps + 7) / 8, (int64_t)sm_count() * 8));
-    if (nch <= 1) cache_row_kernel<T, FMT, BLOCK, S, VEC, 1><<<grid, kThreads, 0, st>>>(x, y, rows, C);
-    else if (nch <= 2) cache_row_kernel<T, FMT, BLOCK, S, VEC, 2><<<grid, kThreads, 0, st>>>(x, y, rows, C);
-    else if (nch <= 3) cache_row_kernel<T, FMT, BLOCK, S, VEC, 3><<<grid, kThreads, 0, st>>>(x, y, rows, C);
-    else if (nch <= 4) cache_row_kernel<T, FMT, BLOCK, S, VEC, 4><<<grid, kThreads, 0, st>>>(x, y, rows, C);
-    else cache_kernel<T, FMT, BLOCK, S, VEC><<<grid, kThreads, 0, st>>>(x, y, rows, C);
+    const int64_t ctas = (warps + kThreads / 32 - 1) / (kThreads / 32);
+    if (nch <= 1) launch_fit_ctas<cache_row_kernel<T, FMT, BLOCK, S, VEC, 1>>(ctas, st, x, y, rows, C);
+    else if (nch <= 2) launch_fit_ctas<cache_row_kernel<T, FMT, BLOCK, S, VEC, 2>>(ctas, st, x, y, rows, C);
+    else if (nch <= 3) launch_fit_ctas<cache_row_kernel<T, FMT, BLOCK, S, VEC, 3>>(ctas, st, x, y, rows, C);
+    else if (nch <= 4) launch_fit_ctas<cache_row_kernel<T, FMT, BLOCK, S, VEC, 4>>(ctas, st, x, y, rows, C);
+    else launch_fit_ctas<cache_kernel<T, FMT, BLOCK, S, VEC>>(ctas, st, x, y, rows, C);
 }
 
 template <typename T, int FMT, int BLOCK, bool VEC>
@@ -242,7 +242,7 @@ static void launch_cache_s(const T* x, T* y, int64_t rows, int64_t C, cudaStream
     const int64_t cpr = ((C + BLOCK - 1) / BLOCK) * (BLOCK / 8);
     if (FMT != BSQ_NVFP4 && VEC && C % BLOCK == 0) {
         const int64_t nchunks = rows * C / 8;
-        cache_flat_kernel<T, FMT, BLOCK, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>(x, y, nchunks);
+        launch_fit<cache_flat_kernel<T, FMT, BLOCK, 4>>(nchunks, 4, st, x, y, nchunks);
         return;
     }
     int S = 2;

@@ -238,6 +238,41 @@ static inline int grid_for(int64_t items, int per_thread) {
     return (int)std::max<int64_t>(1, std::min(need, cap));
 }
 
+// CTAs of KERNEL (kThreads threads, no dynamic shared memory) resident on one
+// SM at once, from the occupancy calculator; cached per device.
+template <auto KERNEL>
+static inline int resident_ctas() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, KERNEL, kThreads, 0) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 1;
+        }
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// Launch a grid-stride KERNEL with one wave of CTAs: enough for `items` at
+// `per_thread` items per thread, and no more than the device holds at once.
+// Every CTA then starts immediately and gets an equal share of the stream,
+// where a grid of several waves leaves SMs idle behind a partial last wave.
+template <auto KERNEL, typename... A>
+static inline void launch_fit_ctas(int64_t ctas_needed, cudaStream_t st, A... args) {
+    const int64_t cap = (int64_t)sm_count() * resident_ctas<KERNEL>();
+    const int grid = (int)std::max<int64_t>(1, std::min(ctas_needed, cap));
+    KERNEL<<<grid, kThreads, 0, st>>>(args...);
+}
+
+template <auto KERNEL, typename... A>
+static inline void launch_fit(int64_t items, int per_thread, cudaStream_t st, A... args) {
+    const int64_t need = (items + (int64_t)kThreads * per_thread - 1) / ((int64_t)kThreads * per_thread);
+    launch_fit_ctas<KERNEL>(need, st, args...);
+}
+
 static inline bsq_status check_dtype(bsq_dtype t) {
     if (t != BSQ_BF16 && t != BSQ_FP32) return fail(BSQ_ERR_UNSUPPORTED, "dtype %d not supported", (int)t);
     return BSQ_OK;

@@ -166,12 +166,12 @@ BSQ_API bsq_status bsq_dequantize_nvfp4(const uint8_t* packed, const uint8_t* sc
     cudaStream_t st = (cudaStream_t)stream;
     if (yt == BSQ_BF16) {
         const int64_t nitems = rows * K / 8;
-        dequant_kernel<FMT_NV, uint16_t, 16, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
-            packed, scales_e4m3, row_scale, bpr, nitems, (uint16_t*)y);
+        launch_fit<dequant_kernel<FMT_NV, uint16_t, 16, 4>>(nitems, 4, st, packed, scales_e4m3, row_scale, bpr, nitems,
+                                                              (uint16_t*)y);
     } else {
         const int64_t nitems = rows * K / 4;
-        dequant_kernel<FMT_NV, float, 16, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
-            packed, scales_e4m3, row_scale, bpr, nitems, (float*)y);
+        launch_fit<dequant_kernel<FMT_NV, float, 16, 4>>(nitems, 4, st, packed, scales_e4m3, row_scale, bpr, nitems,
+                                                           (float*)y);
     }
     return check_launch("bsq_dequantize_nvfp4");
 }
@@ -186,11 +186,10 @@ BSQ_API bsq_status bsq_quantize_mxfp4(const void* x, bsq_dtype xt, int64_t rows,
     const int64_t nchunks = rows * K / 8;
     cudaStream_t st = (cudaStream_t)stream;
     if (xt == BSQ_BF16)
-        flat_quant_kernel<uint16_t, 1, 32, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>((const uint16_t*)x, nchunks,
-                                                                                         packed, scales_e8m0);
+        launch_fit<flat_quant_kernel<uint16_t, 1, 32, 4>>(nchunks, 4, st, (const uint16_t*)x, nchunks, packed,
+                                                            scales_e8m0);
     else
-        flat_quant_kernel<float, 1, 32, 4><<<grid_for(nchunks, 4), kThreads, 0, st>>>((const float*)x, nchunks, packed,
-                                                                                      scales_e8m0);
+        launch_fit<flat_quant_kernel<float, 1, 32, 4>>(nchunks, 4, st, (const float*)x, nchunks, packed, scales_e8m0);
     return check_launch("bsq_quantize_mxfp4");
 }
 
@@ -205,12 +204,12 @@ BSQ_API bsq_status bsq_dequantize_mxfp4(const uint8_t* packed, const uint8_t* sc
     const FastDiv none = make_fastdiv(1);
     if (yt == BSQ_BF16) {
         const int64_t nitems = rows * K / 8;
-        dequant_kernel<FMT_MX, uint16_t, 32, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
-            packed, scales_e8m0, nullptr, none, nitems, (uint16_t*)y);
+        launch_fit<dequant_kernel<FMT_MX, uint16_t, 32, 4>>(nitems, 4, st, packed, scales_e8m0, (const float*)nullptr,
+                                                              none, nitems, (uint16_t*)y);
     } else {
         const int64_t nitems = rows * K / 4;
-        dequant_kernel<FMT_MX, float, 32, 4><<<grid_for(nitems, 4), kThreads, 0, st>>>(
-            packed, scales_e8m0, nullptr, none, nitems, (float*)y);
+        launch_fit<dequant_kernel<FMT_MX, float, 32, 4>>(nitems, 4, st, packed, scales_e8m0, (const float*)nullptr, none,
+                                                           nitems, (float*)y);
     }
     return check_launch("bsq_dequantize_mxfp4");
 }
@@ -224,14 +223,15 @@ BSQ_API bsq_status bsq_quantize_fp8(const void* x, bsq_dtype xt, int64_t rows, i
     if (!codes_e4m3 || !scales_e8m0) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_fp8: null output");
     if (!aligned(x, 16) || !aligned(codes_e4m3, 8)) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_fp8: misaligned pointer");
     const int64_t nchunks = rows * K / 8;
-    const int grid = grid_for(nchunks, 4);
     cudaStream_t st = (cudaStream_t)stream;
     if (xt == BSQ_BF16) {
-        if (block == 32) flat_quant_kernel<uint16_t, 0, 32, 4><<<grid, kThreads, 0, st>>>((const uint16_t*)x, nchunks, codes_e4m3, scales_e8m0);
-        else flat_quant_kernel<uint16_t, 0, 16, 4><<<grid, kThreads, 0, st>>>((const uint16_t*)x, nchunks, codes_e4m3, scales_e8m0);
+        const uint16_t* xb = (const uint16_t*)x;
+        if (block == 32) launch_fit<flat_quant_kernel<uint16_t, 0, 32, 4>>(nchunks, 4, st, xb, nchunks, codes_e4m3, scales_e8m0);
+        else launch_fit<flat_quant_kernel<uint16_t, 0, 16, 4>>(nchunks, 4, st, xb, nchunks, codes_e4m3, scales_e8m0);
     } else {
-        if (block == 32) flat_quant_kernel<float, 0, 32, 4><<<grid, kThreads, 0, st>>>((const float*)x, nchunks, codes_e4m3, scales_e8m0);
-        else flat_quant_kernel<float, 0, 16, 4><<<grid, kThreads, 0, st>>>((const float*)x, nchunks, codes_e4m3, scales_e8m0);
+        const float* xf = (const float*)x;
+        if (block == 32) launch_fit<flat_quant_kernel<float, 0, 32, 4>>(nchunks, 4, st, xf, nchunks, codes_e4m3, scales_e8m0);
+        else launch_fit<flat_quant_kernel<float, 0, 16, 4>>(nchunks, 4, st, xf, nchunks, codes_e4m3, scales_e8m0);
     }
     return check_launch("bsq_quantize_fp8");
 }
@@ -248,11 +248,13 @@ BSQ_API bsq_status bsq_dequantize_fp8(const uint8_t* codes_e4m3, const uint8_t* 
     const FastDiv none = make_fastdiv(1);
     const int64_t nb = rows * K / 8, nf = rows * K / 4;
     if (yt == BSQ_BF16) {
-        if (block == 32) dequant_kernel<FMT_FP8, uint16_t, 32, 4><<<grid_for(nb, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nb, (uint16_t*)y);
-        else dequant_kernel<FMT_FP8, uint16_t, 16, 4><<<grid_for(nb, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nb, (uint16_t*)y);
+        const float* nog = nullptr;
+        if (block == 32) launch_fit<dequant_kernel<FMT_FP8, uint16_t, 32, 4>>(nb, 4, st, codes_e4m3, scales_e8m0, nog, none, nb, (uint16_t*)y);
+        else launch_fit<dequant_kernel<FMT_FP8, uint16_t, 16, 4>>(nb, 4, st, codes_e4m3, scales_e8m0, nog, none, nb, (uint16_t*)y);
     } else {
-        if (block == 32) dequant_kernel<FMT_FP8, float, 32, 4><<<grid_for(nf, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nf, (float*)y);
-        else dequant_kernel<FMT_FP8, float, 16, 4><<<grid_for(nf, 4), kThreads, 0, st>>>(codes_e4m3, scales_e8m0, nullptr, none, nf, (float*)y);
+        const float* nog = nullptr;
+        if (block == 32) launch_fit<dequant_kernel<FMT_FP8, float, 32, 4>>(nf, 4, st, codes_e4m3, scales_e8m0, nog, none, nf, (float*)y);
+        else launch_fit<dequant_kernel<FMT_FP8, float, 16, 4>>(nf, 4, st, codes_e4m3, scales_e8m0, nog, none, nf, (float*)y);
     }
     return check_launch("bsq_dequantize_fp8");
 }

@@ -24,8 +24,11 @@
 //               (bf16x2 multiply), swizzled 16-byte shared stores
 //   warp 20     B producer: TMA loads of 64-token x 64-k activation boxes
 //   warp 21     tensor-memory allocation and the single MMA-issuing thread
-// Tile = 128 features x up to 256 tokens, k-step 64; separate rings of 5
-// dequantized-weight slots (16 KiB) and 4 activation slots (32 KiB);
+// Tile = 128 features x up to 256 tokens, k-step 64; a ring of 4 stages,
+// each a 16 KiB dequantized-weight slot and a 32 KiB activation slot with one
+// full and one empty barrier, so the MMA thread waits once and commits once
+// per k-step (its per-k-step instruction time, not the tensor core, sets the
+// pace of a pipelined loop);
 // two 256-column fp32 accumulators in tensor memory so the epilogue of one
 // tile overlaps the main loop of the next.  Tiles are numbered (expert token
 // tile, feature tile) with the feature tile fastest, dealt round-robin to the
@@ -79,15 +82,18 @@ constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kPrefetch = 4;  // k-steps of packed weights in flight per producer thread
 
 // Shared-memory plan of a CTA group of CG CTAs (1, or a pair with
-// cta_group::2): a ring of dequantized-weight slots and a ring of activation
-// slots; each CTA of a pair holds half of the tile's tokens.
+// cta_group::2): a ring of stages, each the dequantized weight slot of one
+// k-step followed by its activation slot (each CTA of a pair holds half of
+// the tile's tokens).  One "full" barrier per stage collects the producer
+// warps' arrivals and the activation bytes, one "empty" barrier receives the
+// MMA commit: the MMA thread waits once and commits once per k-step.
 template <int CG>
 struct Plan {
-    static constexpr int WSTAGES = (CG == 1) ? 5 : 7;
-    static constexpr int XSTAGES = (CG == 1) ? 4 : 6;
+    static constexpr int STAGES = (CG == 1) ? 4 : 6;
     static constexpr uint32_t kXStage = (TN / CG) * BK * 2;  // 32 KiB or 16 KiB
-    static constexpr size_t kBarOffset = (size_t)WSTAGES * kWStage + (size_t)XSTAGES * kXStage;
-    static constexpr int kNumBars = 2 * WSTAGES + 2 * XSTAGES + 5;
+    static constexpr uint32_t kStage = kWStage + kXStage;    // 48 KiB or 32 KiB
+    static constexpr size_t kBarOffset = (size_t)STAGES * kStage;
+    static constexpr int kNumBars = 2 * STAGES + 5;
     static constexpr size_t kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 +
                                          16 /* tmem slot, flags */ + 4 * (2 * kMaxExperts + 2);
 };
@@ -110,12 +116,9 @@ struct Tile {
 };
 
 struct Shared {
-    uint8_t* w;
-    uint8_t* x;
-    uint64_t* w_full;
-    uint64_t* w_empty;
-    uint64_t* x_full;
-    uint64_t* x_empty;
+    uint8_t* stage;  // stage s: weights at s * kStage, activations kWStage further
+    uint64_t* full;
+    uint64_t* empty;
     uint64_t* acc_full;
     uint64_t* acc_empty;
     uint64_t* drain;
@@ -130,14 +133,11 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
     using P = Plan<CG>;
     Shared s;
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-    s.w = base;
-    s.x = base + P::WSTAGES * kWStage;
+    s.stage = base;
     uint64_t* bars = reinterpret_cast<uint64_t*>(base + P::kBarOffset);
-    s.w_full = bars;
-    s.w_empty = bars + P::WSTAGES;
-    s.x_full = bars + 2 * P::WSTAGES;
-    s.x_empty = bars + 2 * P::WSTAGES + P::XSTAGES;
-    s.acc_full = bars + 2 * P::WSTAGES + 2 * P::XSTAGES;
+    s.full = bars;
+    s.empty = bars + P::STAGES;
+    s.acc_full = bars + 2 * P::STAGES;
     s.acc_empty = s.acc_full + 2;
     s.drain = s.acc_empty + 2;
     s.tmem_slot = reinterpret_cast<uint32_t*>(bars + P::kNumBars);
@@ -236,21 +236,43 @@ struct Unit {
     float g;              // NVFP4 backward row scale
 };
 
-// Forward: unit u = (feature row u / (BK/kUE) of the tile, k segment
-// u % (BK/kUE)).  Backward: unit u = (contraction row u / (WM/kUE) of the
-// k-step, kUE-column segment u % (WM/kUE) of the tile's 128 k columns).
+// Place of unit u in the shared operand tile: its row r and first column c.
+// Forward (K-major, rows = 128 features, columns = 64 k): r = u / (64/kUE).
+// Backward (MN-major, rows = 64 contraction indices, columns = 128 k outputs
+// in two 64-column panels): the eight threads of a quarter-warp take
+// consecutive rows of ONE panel, so their 16-byte stores land on eight
+// different bank groups of the 128-byte swizzle (taking both panels of a row
+// would put two stores on each bank group).
+template <int DIR>
+__device__ __forceinline__ void unit_place(int u, int& r, int& c) {
+    if (DIR == BSQ_FWD) {
+        constexpr int upr = BK / kUE;
+        r = u / upr;
+        c = (u % upr) * kUE;
+    } else {
+        constexpr int upp = 64 / kUE;  // units per row of a panel
+        constexpr int rpq = 8 / upp;   // rows per quarter-warp
+        const int lane = u & 31;
+        r = (u >> 5) * (2 * rpq) + (lane >> 4) * rpq + (lane / upp) % rpq;
+        c = ((lane >> 3) & 1) * 64 + (lane % upp) * kUE;
+    }
+}
+
+// Forward: the unit's row is a feature (weight row), its columns are k.
+// Backward: its row is a contraction index (weight row), its columns are k
+// outputs of the tile.
 template <int FMT, int DIR>
 __device__ __forceinline__ void load_unit(Unit& u, const Args& a, const Tile& ti, int ks, int unit) {
+    int r, c;
+    unit_place<DIR>(unit, r, c);
     int64_t row;
     int kcol;  // first weight column (k) of the unit
     if (DIR == BSQ_FWD) {
-        constexpr int upr = BK / kUE;
-        row = (int64_t)ti.e * a.N + ti.f0 + unit / upr;
-        kcol = ks * BK + (unit % upr) * kUE;
+        row = (int64_t)ti.e * a.N + ti.f0 + r;
+        kcol = ks * BK + c;
     } else {
-        constexpr int upr = WM / kUE;
-        row = (int64_t)ti.e * a.N + ks * BK + unit / upr;
-        kcol = ti.f0 + (unit % upr) * kUE;
+        row = (int64_t)ti.e * a.N + ks * BK + r;
+        kcol = ti.f0 + c;
     }
     const uint8_t* src = a.packed + row * (a.K / 2) + kcol / 2;
     if (kUE == 32) {
@@ -289,18 +311,15 @@ __device__ __forceinline__ void decode_unit(const Unit& u, uint32_t (&v)[kUE / 2
 template <int DIR>
 __device__ __forceinline__ void store_unit(const uint32_t (&v)[kUE / 2], uint32_t w_stage, int unit) {
     // 128-byte shared row of the unit and its first 16-byte chunk in that row
+    int r, col;
+    unit_place<DIR>(unit, r, col);
     uint32_t base;
-    int r, c0;
+    int c0;
     if (DIR == BSQ_FWD) {
-        constexpr int upr = BK / kUE;
-        r = unit / upr;  // K-major: one row per feature, 8-row atoms of 1 KiB
-        c0 = (unit % upr) * (kUE / 8);
+        c0 = col / 8;  // K-major: one row per feature, 8-row atoms of 1 KiB
         base = w_stage + (r >> 3) * 1024 + (r & 7) * 128;
     } else {
-        constexpr int upr = WM / kUE;
-        r = unit / upr;  // MN-major: one row per contraction index, 64-feature panels
-        const int col = (unit % upr) * kUE;
-        c0 = (col % 64) / 8;
+        c0 = (col % 64) / 8;  // MN-major: one row per contraction index, 64-feature panels
         base = w_stage + (col / 64) * (BK * 128) + (r >> 3) * 1024 + (r & 7) * 128;
     }
 #pragma unroll
@@ -331,13 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
     const int group = blockIdx.x / CG, ngroups = gridDim.x / CG;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < P::WSTAGES; ++s) {
-            mbar_init(&sh.w_full[s], kDqWarps * CG);
-            mbar_init(&sh.w_empty[s], 1);
-        }
-        for (int s = 0; s < P::XSTAGES; ++s) {
-            mbar_init(&sh.x_full[s], 1);
-            mbar_init(&sh.x_empty[s], 1);
+        for (int s = 0; s < P::STAGES; ++s) {
+            // every producer warp of the group, plus the leader's activation
+            // producer (its arrive carries the expected bytes)
+            mbar_init(&sh.full[s], kDqWarps * CG + 1);
+            mbar_init(&sh.empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sh.acc_full[i], 1);
@@ -426,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
     } else if (warp < kTmaWarp) {
         // ------------------------------------------------- A (weight) producers
         const int dq = threadIdx.x - kEpiWarps * 32;  // unit index
-        const uint32_t w_base = smem_u32(sh.w);
+        const uint32_t st_base = smem_u32(sh.stage);
         int my_tiles = 0;
         if (num_tiles > group) my_tiles = (num_tiles - 1 - group) / ngroups + 1;
         const int items = my_tiles * k_steps;
@@ -470,14 +487,14 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                             if (lt < num_tiles) lti = cursor_tile(lt);
                         }
                     }
-                    const int s = i % P::WSTAGES;
-                    if (!wait_bar(&sh.w_empty[s], ((i / P::WSTAGES) & 1) ^ 1, sh, args.err)) {
+                    const int s = i % P::STAGES;
+                    if (!wait_bar(&sh.empty[s], ((i / P::STAGES) & 1) ^ 1, sh, args.err)) {
                         ok = false;
                     } else {
-                        store_unit<DIR>(v, w_base + s * kWStage, dq);
+                        store_unit<DIR>(v, st_base + s * P::kStage, dq);
                         fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) arrive_leader<CG>(&sh.w_full[s]);
+                        if (lane == 0) arrive_leader<CG>(&sh.full[s]);
                     }
                 }
             }
@@ -493,20 +510,20 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                 const int half = n_mma / CG;  // this CTA's share of the tokens
                 const int nbox = (half + XBOX - 1) / XBOX;
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
-                    const int s = it % P::XSTAGES;
-                    if (!wait_bar(&sh.x_empty[s], ((it / P::XSTAGES) & 1) ^ 1, sh, args.err)) {
+                    const int s = it % P::STAGES;
+                    if (!wait_bar(&sh.empty[s], ((it / P::STAGES) & 1) ^ 1, sh, args.err)) {
                         ok = false;
                         break;
                     }
-                    uint8_t* dst = sh.x + s * P::kXStage;
+                    uint8_t* dst = sh.stage + s * P::kStage + kWStage;
                     if (CG == 1) {
-                        mbar_arrive_expect_tx(&sh.x_full[s], nbox * kXBoxBytes);
+                        mbar_arrive_expect_tx(&sh.full[s], nbox * kXBoxBytes);
                         for (int b = 0; b < nbox; ++b)
-                            tma_load_2d(dst + b * kXBoxBytes, &tmap_x, &sh.x_full[s], ks * BK, ti.tok0 + b * XBOX);
+                            tma_load_2d(dst + b * kXBoxBytes, &tmap_x, &sh.full[s], ks * BK, ti.tok0 + b * XBOX);
                     } else {
                         // both CTAs' boxes complete on the leader's barrier
-                        if (leader) mbar_arrive_expect_tx(&sh.x_full[s], 2 * nbox * kXBoxBytes);
-                        const uint32_t bar = mapa_shared(smem_u32(&sh.x_full[s]), 0);
+                        if (leader) mbar_arrive_expect_tx(&sh.full[s], 2 * nbox * kXBoxBytes);
+                        const uint32_t bar = mapa_shared(smem_u32(&sh.full[s]), 0);
                         for (int b = 0; b < nbox; ++b)
                             tma_load_2d_pair(dst + b * kXBoxBytes, &tmap_x, bar, ks * BK,
                                              ti.tok0 + (int)rank * half + b * XBOX);
@@ -515,15 +532,21 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
             }
             if (!ok && leader) {
                 // drain the loads still in flight (a pair's loads all count on
-                // the leader's barriers)
-                for (int j = (it > P::XSTAGES ? it - P::XSTAGES : 0); j < it; ++j)
-                    mbar_wait(&sh.x_full[j % P::XSTAGES], (j / P::XSTAGES) & 1, kWaitNs);
+                // the leader's barriers); a stage whose producer warps gave up
+                // never completes, and its wait ends at the time limit, long
+                // after its bytes have landed
+                for (int j = (it > P::STAGES ? it - P::STAGES : 0); j < it; ++j)
+                    mbar_wait(&sh.full[j % P::STAGES], (j / P::STAGES) & 1, kWaitNs);
             }
         }
     } else {
         // ------------------------------------------------ MMA (leader only)
         if (lane == 0 && leader) {
-            const uint32_t w_base = smem_u32(sh.w), x_base = smem_u32(sh.x);
+            const uint32_t st_base = smem_u32(sh.stage);
+            // descriptor advance per 16-wide k slice, in 16-byte units: 32 B
+            // along a K-major row; 16 rows of 128 B (2048 B) of the MN-major
+            // backward weights
+            constexpr uint64_t kAStep = (DIR == BSQ_FWD) ? 2 : 128, kBStep = 2;
             int it = 0, tile_iter = 0;
             bool ok = true;
             for (int t = group; t < num_tiles && ok; t += ngroups, ++tile_iter) {
@@ -535,29 +558,25 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * TN);
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
-                    const int sw = it % P::WSTAGES, sx = it % P::XSTAGES;
-                    if (!wait_bar(&sh.w_full[sw], (it / P::WSTAGES) & 1, sh, args.err) ||
-                        !wait_bar(&sh.x_full[sx], (it / P::XSTAGES) & 1, sh, args.err)) {
+                    const int s = it % P::STAGES;
+                    if (!wait_bar(&sh.full[s], (it / P::STAGES) & 1, sh, args.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t ws = w_base + sw * kWStage, xs = x_base + sx * P::kXStage;
+                    const uint32_t ws = st_base + s * P::kStage;
+                    const uint64_t ad0 = (DIR == BSQ_FWD) ? smem_desc(ws, 16, 1024) : smem_desc(ws, BK * 128, 1024);
+                    const uint64_t bd0 = smem_desc(ws + kWStage, 16, 1024);
 #pragma unroll
                     for (int k16 = 0; k16 < BK / 16; ++k16) {
-                        const uint64_t ad = (DIR == BSQ_FWD) ? smem_desc(ws + k16 * 32, 16, 1024)
-                                                             : smem_desc(ws + k16 * 2048, BK * 128, 1024);
-                        const uint64_t bd = smem_desc(xs + k16 * 32, 16, 1024);
+                        // the start address field (bits 0-13) cannot carry: the
+                        // stage lies below 256 KiB of shared memory
+                        const uint64_t ad = ad0 + kAStep * k16, bd = bd0 + kBStep * k16;
                         if (CG == 1) mma_bf16_ss(d_tmem, ad, bd, idesc, (ks | k16) != 0 ? 1u : 0u);
                         else mma_bf16_ss_pair(d_tmem, ad, bd, idesc, (ks | k16) != 0 ? 1u : 0u);
                     }
-                    if (CG == 1) {
-                        mma_commit(&sh.w_empty[sw]);
-                        mma_commit(&sh.x_empty[sx]);
-                    } else {
-                        mma_commit_pair_multicast(&sh.w_empty[sw], 0x3);
-                        mma_commit_pair_multicast(&sh.x_empty[sx], 0x3);
-                    }
+                    if (CG == 1) mma_commit(&sh.empty[s]);
+                    else mma_commit_pair_multicast(&sh.empty[s], 0x3);
                 }
                 if (ok) {
                     if (CG == 1) mma_commit(&sh.acc_full[acc]);

@@ -162,18 +162,18 @@ static bsq_status launch_nv_rowamax(const T* x, int64_t rows, int64_t K, uint8_t
                                     float* g_out, cudaStream_t st) {
     const int64_t cpr = K / 8;
     if (K <= 65536) {
-        const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * (2048 / kRowThreads));
-        nv_rowamax_quant_kernel<T><<<grid, kRowThreads, 0, st>>>(x, rows, K, packed, scales, g_out);
+        static_assert(kRowThreads == kThreads, "row kernel launched with the common block size");
+        launch_fit_ctas<nv_rowamax_quant_kernel<T>>(rows, st, x, rows, K, packed, scales, g_out);
         return check_launch("bsq_quantize_nvfp4");
     }
     // long rows: amax pass, then the flat pass with the computed row scales
-    const int grid = (int)std::min<int64_t>(rows, (int64_t)sm_count() * 8);
-    row_amax_kernel<T><<<grid, kThreads, 0, st>>>(x, rows, K, g_out);
+    launch_fit_ctas<row_amax_kernel<T>>(rows, st, x, rows, K, g_out);
     BSQ_TRY(check_launch("bsq_quantize_nvfp4"));
     (void)cpr;
     const int64_t nblocks = rows * (K / 16);
-    nv_flat_quant_kernel<T, 2, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
-        x, nblocks, make_fastdiv((uint32_t)(K / 16)), nullptr, nullptr, 0, packed, scales, g_out);
+    const float* none = nullptr;
+    launch_fit<nv_flat_quant_kernel<T, 2, 2>>(nblocks, 2, st, x, nblocks, make_fastdiv((uint32_t)(K / 16)), none, none,
+                                              0, packed, scales, g_out);
     return check_launch("bsq_quantize_nvfp4");
 }
 
@@ -190,11 +190,11 @@ BSQ_API bsq_status bsq_quantize_nvfp4(const void* x, bsq_dtype xt, int64_t rows,
         const int64_t nblocks = rows * (K / 16);
         const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
         if (xt == BSQ_BF16)
-            nv_flat_quant_kernel<uint16_t, 0, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
-                (const uint16_t*)x, nblocks, bpr, row_scale_in, nullptr, 0, packed, scales_e4m3, row_scale_out);
+            launch_fit<nv_flat_quant_kernel<uint16_t, 0, 2>>(nblocks, 2, st, (const uint16_t*)x, nblocks, bpr, row_scale_in,
+                                                             (const float*)nullptr, 0, packed, scales_e4m3, row_scale_out);
         else
-            nv_flat_quant_kernel<float, 0, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
-                (const float*)x, nblocks, bpr, row_scale_in, nullptr, 0, packed, scales_e4m3, row_scale_out);
+            launch_fit<nv_flat_quant_kernel<float, 0, 2>>(nblocks, 2, st, (const float*)x, nblocks, bpr, row_scale_in,
+                                                          (const float*)nullptr, 0, packed, scales_e4m3, row_scale_out);
         return check_launch("bsq_quantize_nvfp4");
     }
     if (xt == BSQ_BF16) return launch_nv_rowamax((const uint16_t*)x, rows, K, packed, scales_e4m3, row_scale_out, st);
@@ -236,13 +236,15 @@ BSQ_API bsq_status bsq_quantize_nvfp4_tensor(const void* x, bsq_dtype xt, int64_
     if (xt == BSQ_BF16) {
         amax_partial_kernel<uint16_t, 4><<<P, kThreads, 0, st>>>((const uint16_t*)x, nchunks, partial);
         BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor"));
-        nv_flat_quant_kernel<uint16_t, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
-            (const uint16_t*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+        launch_fit<nv_flat_quant_kernel<uint16_t, 1, 2>>(nblocks, 2, st, (const uint16_t*)x, nblocks, bpr,
+                                                         (const float*)nullptr, (const float*)partial, P, packed,
+                                                         scales_e4m3, tensor_scale_out);
     } else {
         amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
         BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor"));
-        nv_flat_quant_kernel<float, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
-            (const float*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+        launch_fit<nv_flat_quant_kernel<float, 1, 2>>(nblocks, 2, st, (const float*)x, nblocks, bpr,
+                                                      (const float*)nullptr, (const float*)partial, P, packed,
+                                                      scales_e4m3, tensor_scale_out);
     }
     return check_launch("bsq_quantize_nvfp4_tensor");
 }
@@ -314,13 +316,15 @@ BSQ_API bsq_status bsq_quantize_nvfp4_tensor_noalloc(const void* x, bsq_dtype xt
     if (xt == BSQ_BF16) {
         amax_partial_kernel<uint16_t, 4><<<P, kThreads, 0, st>>>((const uint16_t*)x, nchunks, partial);
         BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
-        nv_flat_quant_kernel<uint16_t, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
-            (const uint16_t*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+        launch_fit<nv_flat_quant_kernel<uint16_t, 1, 2>>(nblocks, 2, st, (const uint16_t*)x, nblocks, bpr,
+                                                         (const float*)nullptr, (const float*)partial, P, packed,
+                                                         scales_e4m3, tensor_scale_out);
     } else {
         amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
         BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
-        nv_flat_quant_kernel<float, 1, 2><<<grid_for(nblocks, 2), kThreads, 0, st>>>(
-            (const float*)x, nblocks, bpr, nullptr, partial, P, packed, scales_e4m3, tensor_scale_out);
+        launch_fit<nv_flat_quant_kernel<float, 1, 2>>(nblocks, 2, st, (const float*)x, nblocks, bpr,
+                                                      (const float*)nullptr, (const float*)partial, P, packed,
+                                                      scales_e4m3, tensor_scale_out);
     }
     return check_launch("bsq_quantize_nvfp4_tensor_noalloc");
 }
