@@ -65,6 +65,8 @@ def lib():
             "o_dequantize_nvfp4": (I32, [P, P, P, I64, I64, P, I32]),
             "o_quantize_mxfp4": (I32, [P, I32, I64, I64, P, P]),
             "o_dequantize_mxfp4": (I32, [P, P, I64, I64, P, I32]),
+            "o_quantize_mxfp8": (I32, [P, I32, I64, I64, P, P]),
+            "o_dequantize_mxfp8": (I32, [P, P, I64, I64, P, I32]),
             "o_quantize_fp8": (I32, [P, I32, I64, I64, I32, P, P]),
             "o_dequantize_fp8": (I32, [P, P, I64, I64, I32, P, I32]),
             "o_quantize_cache": (I32, [I32, I32, P, P, I32, I64, I64]),
@@ -222,6 +224,27 @@ def dequantize_mxfp4(packed, scales, out_dtype=BF16):
     rows = int(np.prod(lead)) if lead else 1
     y = _out(lead + (K,), out_dtype)
     _check(lib().o_dequantize_mxfp4(_p(packed), _p(scales), rows, K, _p(y), out_dtype), "dequantize_mxfp4")
+    return y
+
+
+def quantize_mxfp8(x: np.ndarray):
+    """MXFP8 along the last dim: e4m3 codes [..., K] and e8m0 scales [..., K/32]."""
+    x = np.ascontiguousarray(x)
+    K = x.shape[-1]
+    rows = x.size // K if K else 0
+    codes = np.zeros(x.shape, np.uint8)
+    scales = np.zeros(x.shape[:-1] + (K // 32,), np.uint8)
+    _check(lib().o_quantize_mxfp8(_p(x), _dt(x), rows, K, _p(codes), _p(scales)), "quantize_mxfp8")
+    return codes, scales
+
+
+def dequantize_mxfp8(codes, scales, out_dtype=BF16):
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    K = codes.shape[-1]
+    rows = codes.size // K if K else 0
+    y = _out(codes.shape, out_dtype)
+    _check(lib().o_dequantize_mxfp8(_p(codes), _p(scales), rows, K, _p(y), out_dtype), "dequantize_mxfp8")
     return y
 
 

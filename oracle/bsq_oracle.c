@@ -1,7 +1,7 @@
 /*
  * bsq_oracle.c -- plain, slow, scalar CPU oracle for block-scaled microscaling
- * quantization: NVFP4, MXFP4, FP8 with a power-of-two block scale, and the
- * cache fake-quant.
+ * quantization: NVFP4, MXFP4, MXFP8, FP8 with a power-of-two block scale, and
+ * the cache fake-quant.
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
  * CPU-baseline leg of the benchmark may load this library.  It shares no code,
@@ -25,7 +25,8 @@
  *   [CQ]  "nemo_automodel.components.models.deepseek_v41.quantization":
  *         quantize_cache, _power_of_two_ceiling, _CacheQuantization.
  *   [MO]  ModelOpt "tensor_quantizer.py": _FP8_E4M3_MIN_POSITIVE,
- *         StaticBlockScaleQuantizer._block_scale_from_amax, maxbound.
+ *         StaticBlockScaleQuantizer._block_scale_from_amax, maxbound, is_mxfp
+ *         and _real_quantize (MXFP8: e4m3 elements, one e8m0 scale per 32).
  *
  * Readings where the pages are silent are marked "READING:" and are the same
  * readings the repository's design notes list.
@@ -324,6 +325,50 @@ int o_dequantize_mxfp4(const uint8_t* packed, const uint8_t* scales, int64_t row
     for (int64_t i = 0; i < rows * K; ++i) {
         float v = o_e2m1_val(get_nibble(packed, i));
         float val = v * o_e8m0_val(scales[i / 32]);
+        store_elem(y, dt, i, val);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* MXFP8 ([MO] is_mxfp(8), _real_quantize: num_bits (4, 3), scale_bits        */
+/* (8, 0), block 32)                                                          */
+/* ------------------------------------------------------------------------ */
+
+/* READING: the pages name MXFP8 (e4m3 elements, an e8m0 scale per block of
+ * 32) but do not print its quantize body.  The scale follows [MX]
+ * quantize_mxfp4's rule with the element format's largest binary exponent in
+ * place of e2m1's: 2**(floor(log2(amax)) - 8), since E4M3_MAX = 448 =
+ * 1.75 * 2**8 as E2M1_MAX = 6 = 1.5 * 2**2.  amax == 0 and the e8m0 range
+ * clamp as in MXFP4.  amax / scale lies in [256, 512), so the top of a block
+ * can exceed 448 and saturates there (e4m3_round saturates). */
+static int mxfp8_block_exponent(float amax_b) {
+    int e = (amax_b == 0.0f) ? -127 : o_floor_log2(amax_b) - 8;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+int o_quantize_mxfp8(const void* x, int dt, int64_t rows, int64_t K, uint8_t* codes,
+                     uint8_t* scales) {
+    if (K % 32 != 0) return -1;
+    int64_t nblocks = rows * K / 32;
+    for (int64_t b = 0; b < nblocks; ++b) {
+        int e = mxfp8_block_exponent(block_amax(x, dt, b * 32, 32));
+        scales[b] = (uint8_t)(e + 127);
+        float scale = ldexpf(1.0f, e);
+        for (int j = 0; j < 32; ++j)
+            codes[b * 32 + j] = (uint8_t)o_e4m3_round(load_elem(x, dt, b * 32 + j) / scale);
+    }
+    return 0;
+}
+
+/* value = e4m3 * 2**(scale code - 127). */
+int o_dequantize_mxfp8(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t K,
+                       void* y, int dt) {
+    if (K % 32 != 0) return -1;
+    for (int64_t i = 0; i < rows * K; ++i) {
+        float val = o_e4m3_val(codes[i]) * o_e8m0_val(scales[i / 32]);
         store_elem(y, dt, i, val);
     }
     return 0;

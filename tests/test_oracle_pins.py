@@ -363,6 +363,79 @@ def test_mxfp4_exponent_rule(oracle):
     assert (~nz).sum() == 16
 
 
+# ------------------------------------------------------------- MXFP8 --------
+
+def _mxfp8_requant_closed_form(y):
+    """What requantizing e4m3 * 2**k values must give, from the rule alone:
+    the block maximum m = s * 2**f moves to s * 2**(f - e) with the block
+    exponent e = max(f - 8, -127) (s * 256 unless the e8m0 floor binds); e4m3
+    holds every 4-bit significand up to 448 = 1.75 * 256, so every value
+    returns exactly except values above 448 * 2**e (significand 1.875 at the
+    block's top exponent), which saturate to +-448 * 2**e."""
+    yb = y.astype(np.float64).reshape(-1, 32)
+    m = np.abs(yb).max(axis=1, keepdims=True)
+    f = np.floor(np.log2(np.where(m > 0, m, 1.0)))
+    cap = 448.0 * np.exp2(np.maximum(f - 8, -127))
+    return np.where(np.abs(yb) > cap, np.sign(yb) * cap, yb).reshape(y.shape)
+
+
+def test_mxfp8_round_trip_closed_form(oracle):
+    """e4m3 values times an e8m0 scale, quantized again: exact, except the
+    block-top values with significand 1.875, which saturate to 1.75 * 2**f."""
+    rng = np.random.default_rng(31)
+    R, K = 1024, 512
+    codes = rng.integers(0, 256, (R, K), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x01  # no NaN codes
+    # scale codes up to 246 keep 448 * 2**(code - 127) finite in binary32
+    scales = rng.integers(0, 247, (R, K // 32), dtype=np.uint8)
+    y = oracle.dequantize_mxfp8(codes, scales, out_dtype=oracle.F32)
+    assert np.all(np.isfinite(y))
+    # the dequantized values are exactly e4m3 * 2**k (torch's e4m3 decode)
+    ref = torch_e4m3_decode(codes).astype(np.float64) * np.ldexp(1.0, np.repeat(scales.astype(np.int64) - 127, 32, axis=1))
+    assert np.array_equal(y.astype(np.float64), ref)
+    c2, s2 = oracle.quantize_mxfp8(y)
+    y2 = oracle.dequantize_mxfp8(c2, s2, out_dtype=oracle.F32).astype(np.float64)
+    expect = _mxfp8_requant_closed_form(y)
+    assert np.array_equal(y2, expect)
+    assert (y2 != y).any() and (y2 == y).mean() > 0.99  # both cases occur
+    # bf16 holds e4m3 * 2**k exactly above its subnormal floor
+    yb_scales = np.maximum(scales, 20)
+    yb = oracle.dequantize_mxfp8(codes, yb_scales, out_dtype=oracle.BF16)
+    c3, s3 = oracle.quantize_mxfp8(yb)
+    yb2 = oracle.f32_to_bf16(oracle.dequantize_mxfp8(c3, s3, out_dtype=oracle.F32))
+    assert np.array_equal(yb2, oracle.dequantize_mxfp8(c3, s3, out_dtype=oracle.BF16))
+    assert np.array_equal(oracle.bf16_to_f32(yb2).astype(np.float64),
+                          _mxfp8_requant_closed_form(oracle.bf16_to_f32(yb)))
+
+
+def test_mxfp8_exponent_rule_and_saturation(oracle):
+    """scale = 2**(floor(log2(amax)) - 8): the block maximum lands in
+    [256, 512) before rounding; values above 448 saturate to +-448; the codes
+    below that are torch's e4m3 cast of x / scale; all-zero blocks take
+    scale code 0."""
+    s = _synth()
+    x = s.expert_weights(E=2, N=64, K=512, zero_blocks=8, seed=78)
+    codes, scales = oracle.quantize_mxfp8(x)
+    xf = s.bf16_bits_to_f32(x).reshape(-1, 32)
+    amax = np.abs(xf).max(axis=1)
+    e = scales.reshape(-1).astype(np.int64) - 127
+    nz = amax > 0
+    ratio = amax[nz].astype(np.float64) / np.ldexp(1.0, e[nz])
+    assert np.all((ratio >= 256) & (ratio < 512))
+    assert np.all(scales.reshape(-1)[~nz] == 0) and (~nz).sum() == 16
+    q = (xf.astype(np.float64) / np.ldexp(1.0, e)[:, None]).astype(np.float32)
+    c = codes.reshape(-1, 32)
+    big = np.abs(q) > 448
+    assert big.any()  # the rule does saturate on this data
+    assert np.all(c[big] == np.where(q[big] > 0, 0x7E, 0xFE))
+    assert np.array_equal(c[~big], torch_e4m3(q[~big]))
+    # a block at exactly 500 and 448: both store 448
+    blk = np.zeros((1, 32), np.float32)
+    blk[0, 0], blk[0, 1] = 500.0, -448.0
+    cb, sb = oracle.quantize_mxfp8(blk)
+    assert sb[0, 0] == 127 and cb[0, 0] == 0x7E and cb[0, 1] == 0xFE
+
+
 # ------------------------------------------------------------- FP8 ----------
 
 def test_fp8_pow2_scale_rule(oracle):
