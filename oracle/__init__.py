@@ -65,6 +65,8 @@ def lib():
             "o_dequantize_nvfp4": (I32, [P, P, P, I64, I64, P, I32]),
             "o_quantize_mxfp4": (I32, [P, I32, I64, I64, P, P]),
             "o_dequantize_mxfp4": (I32, [P, P, I64, I64, P, I32]),
+            "o_fake_quantize_nvfp4_static": (I32, [P, I32, I64, I64, P, F, P]),
+            "o_nvfp4_static_scale": (None, [F, F, P, P]),
             "o_quantize_mxfp8": (I32, [P, I32, I64, I64, P, P]),
             "o_dequantize_mxfp8": (I32, [P, P, I64, I64, P, I32]),
             "o_quantize_fp8": (I32, [P, I32, I64, I64, I32, P, P]),
@@ -225,6 +227,28 @@ def dequantize_mxfp4(packed, scales, out_dtype=BF16):
     y = _out(lead + (K,), out_dtype)
     _check(lib().o_dequantize_mxfp4(_p(packed), _p(scales), rows, K, _p(y), out_dtype), "dequantize_mxfp4")
     return y
+
+
+def fake_quantize_nvfp4_static(x: np.ndarray, block_amax: np.ndarray, global_amax: float):
+    """Static two-level NVFP4 fake-quant along the last dim (K % 16 == 0) with
+    calibrated per-16-block amax [..., K/16] and a global amax; same dtype as x."""
+    x = np.ascontiguousarray(x)
+    K = x.shape[-1]
+    rows = x.size // K if K else 0
+    a = np.ascontiguousarray(block_amax, dtype=np.float32)
+    assert a.size == rows * (K // 16), "one amax per 16-block"
+    y = np.empty_like(x)
+    _check(lib().o_fake_quantize_nvfp4_static(_p(x), _dt(x), rows, K, _p(a), float(global_amax), _p(y)),
+           "fake_quantize_nvfp4_static")
+    return y
+
+
+def nvfp4_static_scale(amax_b: float, global_amax: float):
+    """(physical block scale, e4m3 code) of one block of the static rule."""
+    sq = ctypes.c_float()
+    code = ctypes.c_int()
+    lib().o_nvfp4_static_scale(float(amax_b), float(global_amax), ctypes.byref(sq), ctypes.byref(code))
+    return sq.value, code.value
 
 
 def quantize_mxfp8(x: np.ndarray):

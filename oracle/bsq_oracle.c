@@ -1,7 +1,7 @@
 /*
  * bsq_oracle.c -- plain, slow, scalar CPU oracle for block-scaled microscaling
- * quantization: NVFP4, MXFP4, MXFP8, FP8 with a power-of-two block scale, and
- * the cache fake-quant.
+ * quantization: NVFP4, MXFP4, MXFP8, FP8 with a power-of-two block scale, the
+ * cache fake-quant and the static two-level NVFP4 fake-quant.
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
  * CPU-baseline leg of the benchmark may load this library.  It shares no code,
@@ -282,6 +282,58 @@ int o_dequantize_nvfp4(const uint8_t* packed, const uint8_t* scales, const float
             float prod = v * s;
             float val = prod * g[r];
             store_elem(y, dt, r * K + k, val);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Static two-level NVFP4 fake-quant ([MO] StaticBlockScaleQuantizer:        */
+/* _block_scale_from_amax with quantize=True, _amax_to_scale, _clamp_scale,  */
+/* _fake_quantize)                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* Calibrated per-16-block amax and a global amax (both given):
+ *   per_tensor_scale pts = _amax_to_scale(global_amax, 6)
+ *                        = A/6, or 1e-8 where A/6 <= 1e-8
+ *   min_value = (E4M3 smallest subnormal / 448) * pts
+ *   scale_b   = _amax_to_scale(amax_b, 6, min_value)
+ *             = amax_b/6, or min_value where amax_b/6 <= min_value
+ *   scale_q   = scaled_e4m3(scale_b, pts): scale_b as an e4m3 number in the
+ *               units that map pts to 448
+ *   y         = cast(e2m1(x / scale_q) * scale_q)
+ * binary32 throughout; Python float constants enter as binary32 (torch
+ * evaluates a float32 tensor op with a Python scalar in float32).
+ * READING: the pages print neither scaled_e4m3 nor
+ * static_blockwise_fp4_fake_quant.  Per the comment at min_value, scaled_e4m3
+ * maps pts to 448: f = 448 / pts, code = e4m3(scale_b * f), and the same map
+ * inverted gives the physical scale, scale_q = e4m3 value / f.  The static
+ * path is taken to compute what the LSQ path prints with pre = post amax. */
+void o_nvfp4_static_scale(float amax_b, float global_amax, float* scale_q, int* code) {
+    const float one_e8 = 1e-8f;
+    float pts = global_amax / 6.0f;
+    if (pts <= one_e8) pts = one_e8;
+    const float c0 = (float)(E4M3_MIN_SUBNORMAL / 448.0);
+    const float min_value = c0 * pts;
+    float sb = amax_b / 6.0f;
+    if (sb <= min_value) sb = min_value;
+    const float f = 448.0f / pts;
+    *code = o_e4m3_round(sb * f);
+    *scale_q = o_e4m3_val(*code) / f;
+}
+
+int o_fake_quantize_nvfp4_static(const void* x, int dt, int64_t rows, int64_t K,
+                                 const float* block_amax, float global_amax, void* y) {
+    if (K % 16 != 0) return -1;
+    int64_t nblocks = rows * K / 16;
+    for (int64_t b = 0; b < nblocks; ++b) {
+        float scale_q;
+        int code;
+        o_nvfp4_static_scale(block_amax[b], global_amax, &scale_q, &code);
+        for (int j = 0; j < 16; ++j) {
+            float q = load_elem(x, dt, b * 16 + j) / scale_q;
+            float w = o_e2m1_val(o_e2m1_round(q));
+            store_elem(y, dt, b * 16 + j, w * scale_q);
         }
     }
     return 0;

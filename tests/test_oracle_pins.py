@@ -363,6 +363,71 @@ def test_mxfp4_exponent_rule(oracle):
     assert (~nz).sum() == 16
 
 
+# ------------------------------------------------- static two-level NVFP4 --
+
+def _block_amax(xf, block=16):
+    return np.abs(xf.reshape(-1, block)).max(axis=1).astype(np.float32)
+
+
+def test_nvfp4_static_reduces_to_per_row_nvfp4(oracle):
+    """With the block amax calibrated to the data and a global amax of
+    2688 * 2**k (so A/6 and 448/(A/6) are exact), the static two-level rule
+    is the NVFP4 rule with row scale g = 2**k: bit-identical to the pinned
+    quantize_nvfp4(x, row_scale=2**k) -> dequantize_nvfp4 round trip."""
+    s = _synth()
+    x = s.nvfp4_matrix(rows=64, cols=512, seed=91)
+    xf = s.bf16_bits_to_f32(x)
+    for k in (-6, 0, 3):
+        A = np.float32(2688.0 * 2.0 ** k)
+        y = oracle.fake_quantize_nvfp4_static(x, _block_amax(xf), A)
+        p, sc, g = oracle.quantize_nvfp4(x, row_scale=np.float32(2.0 ** k))
+        assert np.array_equal(y, oracle.dequantize_nvfp4(p, sc, g)), k
+        y32 = oracle.fake_quantize_nvfp4_static(xf, _block_amax(xf), A)
+        assert np.array_equal(y32, oracle.dequantize_nvfp4(*oracle.quantize_nvfp4(xf, row_scale=np.float32(2.0 ** k)),
+                                                           out_dtype=oracle.F32)), k
+
+
+def test_nvfp4_static_is_nearest_multiple(oracle, golden_dir):
+    """Every output is the nearest of the 16 e2m1 values times the block's
+    physical scale (brute force in float64, ties to the even code, values past
+    6 saturate), for calibrated amax below, at and above the data's."""
+    s = _synth()
+    x = s.nvfp4_matrix(rows=32, cols=256, seed=92)
+    xf = s.bf16_bits_to_f32(x)
+    table = e2m1_table_golden(golden_dir)
+    rng = np.random.default_rng(93)
+    amax = _block_amax(xf) * rng.choice([0.25, 1.0, 3.0], size=xf.size // 16).astype(np.float32)
+    A = np.float32(np.abs(xf).max() * 1.5)
+    y = oracle.fake_quantize_nvfp4_static(xf, amax, A)
+    sq = np.array([oracle.nvfp4_static_scale(a, A)[0] for a in amax], np.float64)
+    q = (xf.reshape(-1, 16).astype(np.float64) / sq[:, None]).astype(np.float32)
+    codes = brute_e2m1(q.reshape(-1), table).reshape(-1, 16)
+    vals = np.where(codes >= 8, -1.0, 1.0) * table[codes & 7]
+    want = (vals * sq[:, None]).astype(np.float32)
+    assert np.array_equal(y.reshape(-1, 16), want)
+    # calibrated amax at a quarter of the data's: the block maxima saturate
+    low = amax < _block_amax(xf)
+    assert np.all(np.abs(y.reshape(-1, 16)[low]).max(axis=1) == (6.0 * sq[low]).astype(np.float32))
+
+
+def test_nvfp4_static_scale_floor_and_range(oracle):
+    """The physical scale is within e4m3 precision of amax/6, never below the
+    e4m3 floor 2**-9 * A/2688, and a zero amax lands exactly on that floor."""
+    rng = np.random.default_rng(94)
+    A = np.float32(37.5)
+    unit = np.float64(A) / 6 / 448
+    for a in np.exp(rng.uniform(np.log(1e-6), np.log(37.5), 2000)).astype(np.float32):
+        sq, code = oracle.nvfp4_static_scale(a, A)
+        assert sq >= 2.0 ** -9 * unit * (1 - 1e-6)
+        if np.float64(a) / 6 >= 2.0 ** -6 * unit:  # the e4m3 normal range: 3 mantissa bits
+            assert abs(sq / (np.float64(a) / 6) - 1) <= 2.0 ** -4 * (1 + 1e-6)
+    sq0, code0 = oracle.nvfp4_static_scale(0.0, A)
+    assert code0 == 1 and abs(sq0 / (2.0 ** -9 * unit) - 1) < 1e-6
+    # a zero global amax falls back to the 1e-8 per-tensor floor
+    sqz, codez = oracle.nvfp4_static_scale(0.0, 0.0)
+    assert codez == 1 and abs(sqz / (2.0 ** -9 * 1e-8 / 448) - 1) < 1e-6
+
+
 # ------------------------------------------------------------- MXFP8 --------
 
 def _mxfp8_requant_closed_form(y):
