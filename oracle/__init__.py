@@ -66,6 +66,7 @@ def lib():
             "o_quantize_mxfp4": (I32, [P, I32, I64, I64, P, P]),
             "o_dequantize_mxfp4": (I32, [P, P, I64, I64, P, I32]),
             "o_fake_quantize_nvfp4_static": (I32, [P, I32, I64, I64, P, F, P]),
+            "o_dequantize_kv_cache_nvfp4": (I32, [P, P, P, I64, I64, I64, P, I32]),
             "o_nvfp4_static_scale": (None, [F, F, P, P]),
             "o_quantize_mxfp8": (I32, [P, I32, I64, I64, P, P]),
             "o_dequantize_mxfp8": (I32, [P, P, I64, I64, P, I32]),
@@ -226,6 +227,25 @@ def dequantize_mxfp4(packed, scales, out_dtype=BF16):
     rows = int(np.prod(lead)) if lead else 1
     y = _out(lead + (K,), out_dtype)
     _check(lib().o_dequantize_mxfp4(_p(packed), _p(scales), rows, K, _p(y), out_dtype), "dequantize_mxfp4")
+    return y
+
+
+def dequantize_kv_cache_nvfp4(values, scales, amax, block_tokens: int, heads: int, out_dtype=BF16):
+    """List-of-blocks NVFP4 KV cache -> [1, nblocks * block_tokens, heads, 128].
+    values[b] uint8 [block_tokens * heads, 64], scales[b] uint8 [.., 8],
+    amax float32 [nblocks] (one per block)."""
+    nb = len(values)
+    rows = block_tokens * heads
+    vals = [np.ascontiguousarray(v, dtype=np.uint8) for v in values]
+    scs = [np.ascontiguousarray(s_, dtype=np.uint8) for s_ in scales]
+    for v, s_ in zip(vals, scs):
+        assert v.shape == (rows, 64) and s_.shape == (rows, 8)
+    vp = (ctypes.c_void_p * max(nb, 1))(*[v.ctypes.data for v in vals])
+    sp = (ctypes.c_void_p * max(nb, 1))(*[s_.ctypes.data for s_ in scs])
+    am = np.ascontiguousarray(amax, dtype=np.float32)
+    y = _out((1, nb * block_tokens, heads, 128), out_dtype)
+    _check(lib().o_dequantize_kv_cache_nvfp4(vp, sp, _p(am), nb, block_tokens, heads, _p(y), out_dtype),
+           "dequantize_kv_cache_nvfp4")
     return y
 
 

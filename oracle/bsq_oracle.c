@@ -24,6 +24,9 @@
  *         _FP4_E2M1_MIDPOINTS, _FP4_BYTE_TABLE, MXFP4_BLOCK_SIZE.
  *   [CQ]  "nemo_automodel.components.models.deepseek_v41.quantization":
  *         quantize_cache, _power_of_two_ceiling, _CacheQuantization.
+ *   [KV]  "nemo_automodel ... quantization" model-filter page:
+ *         dequantize_kv_cache, _dequantize_kv_cache_fused_cuda (the
+ *         list-of-blocks NVFP4 KV cache and its contiguous output layout).
  *   [MO]  ModelOpt "tensor_quantizer.py": _FP8_E4M3_MIN_POSITIVE,
  *         StaticBlockScaleQuantizer._block_scale_from_amax, maxbound, is_mxfp
  *         and _real_quantize (MXFP8: e4m3 elements, one e8m0 scale per 32).
@@ -284,6 +287,37 @@ int o_dequantize_nvfp4(const uint8_t* packed, const uint8_t* scales, const float
             store_elem(y, dt, r * K + k, val);
         }
     }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Paged NVFP4 KV cache ([KV] dequantize_kv_cache)                          */
+/* ------------------------------------------------------------------------ */
+
+/* A list of nblocks quantized blocks; block b holds block_tokens * heads rows
+ * of 128 values (row = token-in-block * heads + head): e2m1 codes
+ * values[b] [rows, 64], e4m3 scales scales[b] [rows, 8] and one amax[b].
+ * Its global scale is amax[b] / (6 * 448) (the scale rule's e2m1 and e4m3
+ * maxima) and its rows dequantize as in dequantize_nvfp4.  Output
+ * [1, nblocks * block_tokens, heads, 128]: token t of block b is output token
+ * b * block_tokens + t.
+ * READING: from_blocked (the swizzled scale layout) is not on the pages, so
+ * the scales are the row-major [rows, 8] layout the other NVFP4 functions use. */
+int o_dequantize_kv_cache_nvfp4(const uint8_t* const* values, const uint8_t* const* scales,
+                                const float* amax, int64_t nblocks, int64_t block_tokens,
+                                int64_t heads, void* y, int dt) {
+    const int64_t rows = block_tokens * heads;
+    const int elem = (dt == O_BF16) ? 2 : 4;
+    float* g = (float*)malloc(sizeof(float) * (size_t)(rows > 0 ? rows : 1));
+    if (!g) return -2;
+    for (int64_t b = 0; b < nblocks; ++b) {
+        const float gb = amax[b] / (E2M1_MAX * E4M3_MAX);
+        for (int64_t r = 0; r < rows; ++r) g[r] = gb;
+        /* block b's rows are the contiguous output range starting at token b * block_tokens */
+        void* yb = (char*)y + (size_t)(b * rows * 128) * (size_t)elem;
+        o_dequantize_nvfp4(values[b], scales[b], g, rows, 128, yb, dt);
+    }
+    free(g);
     return 0;
 }
 

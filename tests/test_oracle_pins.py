@@ -363,6 +363,39 @@ def test_mxfp4_exponent_rule(oracle):
     assert (~nz).sum() == 16
 
 
+# ------------------------------------------------------- paged KV cache ----
+
+def test_kv_cache_layout_and_values(oracle, golden_dir):
+    """Output [1, blocks * block_tokens, heads, 128]: element (b * bt + t, h, d)
+    is code d of row t * heads + h of block b, times that row's e4m3 scale for
+    column d // 16, times the block's amax / 2688 -- assembled here from the
+    printed e2m1 table, torch's e4m3 decode and binary32 products."""
+    rng = np.random.default_rng(71)
+    nb, bt, heads = 5, 4, 3
+    rows = bt * heads
+    vals = [rng.integers(0, 256, (rows, 64), dtype=np.uint8) for _ in range(nb)]
+    scs = []
+    for _ in range(nb):
+        sc = rng.integers(0, 127, (rows, 8), dtype=np.uint8)  # finite, non-negative e4m3
+        scs.append(sc)
+    amax = np.array([2688.0, 1.0, 0.0, 3.5e5, 7e-3], np.float32)
+    table = e2m1_table_golden(golden_dir).astype(np.float32)
+    for dt in (oracle.BF16, oracle.F32):
+        y = oracle.dequantize_kv_cache_nvfp4(vals, scs, amax, bt, heads, out_dtype=dt)
+        assert y.shape == (1, nb * bt, heads, 128)
+        yf = oracle.bf16_to_f32(y) if dt == oracle.BF16 else y
+        for b in range(nb):
+            g = np.float32(amax[b]) / np.float32(2688.0)
+            codes = np.stack([vals[b] & 15, vals[b] >> 4], axis=-1).reshape(rows, 128)
+            e2 = np.where(codes >= 8, -1.0, 1.0).astype(np.float32) * table[codes & 7]
+            sv = np.repeat(torch_e4m3_decode(scs[b]).astype(np.float32), 16, axis=1)
+            want = (e2 * sv).astype(np.float32) * g
+            if dt == oracle.BF16:
+                want = oracle.bf16_to_f32(oracle.f32_to_bf16(want))
+            got = yf[0, b * bt:(b + 1) * bt].reshape(rows, 128)  # row = t * heads + h
+            assert np.array_equal(got, want), (b, dt)
+
+
 # ------------------------------------------------- static two-level NVFP4 --
 
 def _block_amax(xf, block=16):
