@@ -13,10 +13,12 @@ per second over the timed region, summed over ranks (weak scaling: each rank
 runs its own copy of the workload; the path has no data exchange).
 
 The same run also times the other workloads as sub-measurements ("extra"):
-NVFP4 [256, 2048] round trip latency, the cache fake-quant cases, the
+NVFP4 [256, 2048] round trip latency, MXFP8 quantize / dequantize of the
+same [8, 2048, 7168] expert weights, the list-of-blocks NVFP4 KV-cache
+dequantize (1024 blocks of 64 tokens x 8 heads), the cache fake-quant cases, the
 [7168, 18432] NVFP4 weight quantization (ModelOpt per-tensor, per-row,
-gate/up) and the fused-dequant grouped GEMM (TFLOP/s), each with its HBM or
-tensor roofline.
+gate/up, the static two-level fake-quant) and the fused-dequant grouped GEMM
+(TFLOP/s), each with its HBM or tensor roofline.
 
 --impl reference times the CPU oracle (the only reference this path has) on a
 bounded sample of the same workload on the host cores.
@@ -50,8 +52,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the sub-measurements of the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
-    ap.add_argument("--only", default="", help="run only these sub-measurements (comma list of nvfp4,cache,linear,"
-                    "gemm) and print them, without the main step; for profiling")
+    ap.add_argument("--only", default="", help="run only these sub-measurements (comma list of nvfp4,mxfp8,kv,"
+                    "cache,linear,gemm) and print them, without the main step; for profiling")
     ap.add_argument("--gemm-only", default="", help="time only these grouped-GEMM variants (comma list of "
                     "mxfp4_fwd,mxfp4_bwd,nvfp4_fwd,nvfp4_bwd) and print them; for profiling")
     return ap.parse_args()
@@ -71,6 +73,8 @@ KERNEL_SOURCES = {
     "flat": ["flat.cu", "common.cuh", "formats.cuh", "host_util.h"],
     "nvfp4": ["nvfp4.cu", "common.cuh", "formats.cuh", "host_util.h"],
     "cache": ["cache.cu", "common.cuh", "formats.cuh", "host_util.h"],
+    "static": ["static.cu", "common.cuh", "formats.cuh", "host_util.h"],
+    "kv": ["kv_cache.cu", "common.cuh", "formats.cuh", "host_util.h"],
     "gemm": ["grouped_mm.cu", "tcgen05.cuh", "formats.cuh", "host_util.h"],
 }
 
@@ -488,6 +492,39 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
             "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_nvfp4(p, s, r, y=y), 50, True), nb),
             "note": "latency-bound (1.3 MB); L2 flushed before every launch"}
 
+    if want("mxfp8"):
+        g = torch.Generator(device=dev)
+        g.manual_seed(20260006)
+        x = synth.expert_weights_torch(E, N, K, generator=g, device=dev)
+        n = x.numel()
+        c = torch.empty((E, N, K), dtype=torch.uint8, device=dev)
+        s = torch.empty((E, N, K // 32), dtype=torch.uint8, device=dev)
+        y = torch.empty_like(x)
+        out["mxfp8_expert_weights_8x2048x7168"] = {
+            "quantize": rec(timed(lambda: bsq.bsq_quantize_mxfp8(x, codes=c, scales=s), 10, False),
+                            2 * n + n + n // 32, "mxfp8_quant"),
+            "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_mxfp8(c, s, y=y), 10, False),
+                                   n + n // 32 + 2 * n, "mxfp8_dequant_bf16"),
+            "note": "inputs and outputs larger than L2"}
+        del x, c, s, y
+
+    if want("kv"):
+        g = torch.Generator(device=dev)
+        g.manual_seed(20260007)
+        nbk, bt, hd = 1024, 64, 8
+        rows = bt * hd
+        vals = [torch.randint(0, 256, (rows, 64), generator=g, device=dev, dtype=torch.uint8) for _ in range(nbk)]
+        scs = [torch.randint(0, 0x7E, (rows, 8), generator=g, device=dev, dtype=torch.uint8) for _ in range(nbk)]
+        ams = [torch.rand((1,), generator=g, device=dev) * 100 for _ in range(nbk)]
+        table = bsq.kv_block_table(vals, scs, ams)
+        yk = torch.empty((1, nbk * bt, hd, 128), dtype=torch.bfloat16, device=dev)
+        n = nbk * rows * 128
+        out["kv_cache_nvfp4_1024x64x8x128"] = {
+            "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_kv_cache_nvfp4(table, nbk, bt, hd, y=yk), 10, True),
+                                   n // 2 + n // 16 + 4 * nbk + 2 * n, "kv_dequant_bf16"),
+            "note": "1024 separately allocated blocks of 64 tokens x 8 heads x 128; L2 flushed before every launch"}
+        del vals, scs, ams, table, yk
+
     if want("cache"):
         g = torch.Generator(device=dev)
         g.manual_seed(20260003)
@@ -530,6 +567,10 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
         nb_gu = 2 * (2 * n) + (2 * n) // 2 + (2 * n) // 16 + 2 * 4 * 14336
         y = torch.empty((7168, 18432), dtype=torch.bfloat16, device=dev)
         nb_dq = n // 2 + n // 16 + 4 * 7168 + 2 * n
+        # static two-level fake-quant: calibrated block amax = the data's own
+        bam = x.view(-1, 16).abs().amax(dim=1).float()
+        gam = x.abs().amax().float().reshape(1)
+        nb_st = 2 * n + 4 * (n // 16) + 2 * n
         out["nvfp4_linear_7168x18432"] = {
             "modelopt_tensor_scale": rec(timed(lambda: bsq.bsq_quantize_nvfp4_tensor(
                 x, packed=p, scales=s, tensor_scale=t, scratch=scratch), 10, False), nb_tensor,
@@ -541,6 +582,8 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
                 "nvfp4_gate_up_given_row_scales"),
             "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_nvfp4(p, s, r, y=y), 10, False), nb_dq,
                                    "nvfp4_dequant_bf16"),
+            "static_two_level_fake_quant": rec(timed(lambda: bsq.bsq_fake_quantize_nvfp4_static(x, bam, gam, y=y),
+                                                     10, False), nb_st, "nvfp4_static_fake_quant"),
             "note": "inputs larger than L2; per-tensor counts two reads of the input"}
         del x, cat, y
 

@@ -36,6 +36,7 @@ class Format(enum.IntEnum):
     FP8 = 0
     MXFP4 = 1
     NVFP4 = 2
+    MXFP8 = 3
 
 
 class Direction(enum.IntEnum):
@@ -65,6 +66,10 @@ _SIGS = {
     "bsq_dequantize_nvfp4": (_I32, [_P, _P, _P, _I64, _I64, _P, _I32, _P]),
     "bsq_quantize_mxfp4": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P]),
     "bsq_dequantize_mxfp4": (_I32, [_P, _P, _I64, _I64, _P, _I32, _P]),
+    "bsq_fake_quantize_nvfp4_static": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _P]),
+    "bsq_dequantize_kv_cache_nvfp4": (_I32, [_P, _P, _P, _I64, _I64, _I64, _P, _I32, _P]),
+    "bsq_quantize_mxfp8": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P]),
+    "bsq_dequantize_mxfp8": (_I32, [_P, _P, _I64, _I64, _P, _I32, _P]),
     "bsq_quantize_fp8": (_I32, [_P, _I32, _I64, _I64, _I32, _P, _P, _P]),
     "bsq_dequantize_fp8": (_I32, [_P, _P, _I64, _I64, _I32, _P, _I32, _P]),
     "bsq_quantize_cache": (_I32, [_I32, _I32, _P, _P, _I32, _I64, _I64, _P]),
@@ -217,6 +222,54 @@ def bsq_dequantize_mxfp4(packed, scales, out_dtype=DType.BF16, y=None, stream=No
 
 
 # -------------------------------------------------------------------- FP8 ---
+
+def kv_block_table(values, scales, amax, device=None):
+    """Device arrays of the blocks' pointers for bsq_dequantize_kv_cache_nvfp4
+    (lists of uint8 [rows, 64] codes, uint8 [rows, 8] scales and fp32 [1] amax
+    tensors).  Build once per cache layout; the tensors must stay alive."""
+    dev_ = device if device is not None else values[0].device
+    def table(ts):
+        return torch.tensor([t.data_ptr() for t in ts], dtype=torch.int64).to(dev_)
+    return table(values), table(scales), table(amax)
+
+
+def bsq_dequantize_kv_cache_nvfp4(table, nblocks, block_tokens, heads, out_dtype=DType.BF16, y=None, stream=None):
+    """Dequantize a list-of-blocks NVFP4 KV cache into [1, nblocks * block_tokens,
+    heads, 128]; `table` is the (values, scales, amax) pointer arrays of
+    kv_block_table."""
+    vt, st_, at = table
+    if y is None:
+        y = torch.empty((1, nblocks * block_tokens, heads, 128), dtype=_torch_dtype(out_dtype), device=vt.device)
+    _call("bsq_dequantize_kv_cache_nvfp4", _ptr(vt), _ptr(st_), _ptr(at), int(nblocks), int(block_tokens), int(heads),
+          _ptr(y), _dtype_of(y), _stream(stream))
+    return y
+
+
+def bsq_fake_quantize_nvfp4_static(x, block_amax, global_amax, y=None, stream=None):
+    """Static two-level NVFP4 fake-quant: block_amax fp32 [..., K/16] and
+    global_amax fp32 [1] on the device; returns y (x's dtype; y may be x)."""
+    rows, K = _rows_k(x)
+    y = torch.empty_like(x) if y is None else y
+    _call("bsq_fake_quantize_nvfp4_static", _ptr(x), _dtype_of(x), rows, K, _ptr(block_amax), _ptr(global_amax),
+          _ptr(y), _stream(stream))
+    return y
+
+
+def bsq_quantize_mxfp8(x, codes=None, scales=None, stream=None):
+    rows, K = _rows_k(x)
+    lead = tuple(x.shape[:-1])
+    codes = _empty(tuple(x.shape), torch.uint8, x) if codes is None else codes
+    scales = _empty(lead + (K // 32,), torch.uint8, x) if scales is None else scales
+    _call("bsq_quantize_mxfp8", _ptr(x), _dtype_of(x), rows, K, _ptr(codes), _ptr(scales), _stream(stream))
+    return codes, scales
+
+
+def bsq_dequantize_mxfp8(codes, scales, out_dtype=DType.BF16, y=None, stream=None):
+    rows, K = _rows_k(codes)
+    y = _empty(tuple(codes.shape), _torch_dtype(out_dtype), codes) if y is None else y
+    _call("bsq_dequantize_mxfp8", _ptr(codes), _ptr(scales), rows, K, _ptr(y), _dtype_of(y), _stream(stream))
+    return y
+
 
 def bsq_quantize_fp8(x, block=32, codes=None, scales=None, stream=None):
     rows, K = _rows_k(x)

@@ -18,7 +18,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libbsq.so")
-SOURCES = ["abi.cu", "flat.cu", "nvfp4.cu", "cache.cu", "grouped_mm.cu"]
+SOURCES = ["abi.cu", "flat.cu", "nvfp4.cu", "static.cu", "kv_cache.cu", "cache.cu", "grouped_mm.cu"]
 HEADERS = ["common.cuh", "formats.cuh", "host_util.h", "tcgen05.cuh"]
 
 NVCC_FLAGS = [
@@ -49,18 +49,32 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
+def _wait_all(procs):
+    failed = [p.args for p in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, failed[0])
+
+
 def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
+    """Compile every source (in parallel, one nvcc per file) and link."""
     if not force and up_to_date():
         return LIB
-    objs = []
+    objs, cmds = [], []
     for src in SOURCES:
         obj = os.path.join(CSRC, src.replace(".cu", f".{os.getpid()}.o"))
-        cmd = [nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", os.path.join(ROOT, "include"), "-c",
-               os.path.join(CSRC, src), "-o", obj]
+        cmds.append([nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", os.path.join(ROOT, "include"), "-c",
+                     os.path.join(CSRC, src), "-o", obj])
+        objs.append(obj)
+    jobs = max(1, min(len(cmds), os.cpu_count() or 1))
+    running = []
+    for cmd in cmds:
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.check_call(cmd)
-        objs.append(obj)
+        running.append(subprocess.Popen(cmd))
+        if len(running) >= jobs:
+            _wait_all(running[:1])
+            running = running[1:]
+    _wait_all(running)
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp]
     if verbose:

@@ -104,6 +104,13 @@ __device__ __forceinline__ int mx_exponent(float amax_b) {
     return max(-127, min(127, e));
 }
 
+// MXFP8 block exponent: the MXFP4 rule with e4m3's largest exponent,
+// floor(log2(amax)) - 8 (448 = 1.75 * 2**8), zero block -127, clamped.
+__device__ __forceinline__ int mx8_exponent(float amax_b) {
+    int e = (amax_b == 0.0f) ? -127 : floor_log2_exact(amax_b) - 8;
+    return max(-127, min(127, e));
+}
+
 // Power-of-two block scale pow2ceil(max(amax / fmt_max, 2**-126)).
 __device__ __forceinline__ float pow2_scale(float amax_b, float fmt_max) {
     float a = __fdiv_rn(amax_b, fmt_max);

@@ -1,4 +1,4 @@
-// flat.cu -- MXFP4 and FP8 (power-of-two) quantize, and dequantize for all formats.
+// flat.cu -- MXFP4, MXFP8 and FP8 (power-of-two) quantize, and dequantize for all formats.
 //
 // Work unit: a "chunk" of 8 consecutive elements (one 16-byte bf16 vector).
 // A 16- or 32-column block spans 2 or 4 adjacent lanes of a warp, so the
@@ -8,7 +8,9 @@
 //
 // Formulas: mxfp4 page quantize_mxfp4 / dequantize_mxfp4; nvfp4 page
 // dequantize_nvfp4; deepseek_v41 quantization page quantize_cache ("fp8"),
-// _power_of_two_ceiling.
+// _power_of_two_ceiling; ModelOpt tensor_quantizer page, is_mxfp /
+// _real_quantize (MXFP8: e4m3 elements, e8m0 scale per 32), with the MXFP4
+// exponent rule carried over to e4m3 (2**(floor(log2(amax)) - 8)).
 #include <cstdarg>
 #include <cstring>
 #include <mutex>
@@ -21,7 +23,7 @@ namespace bsq {
 // ----------------------------------------------------------- MXFP4 / FP8 ----
 // Flat block quantization (blocks never cross rows because K % block == 0).
 
-template <typename T, int FMT /*0 = fp8, 1 = mxfp4*/, int BLOCK, int U>
+template <typename T, int FMT /*0 = fp8, 1 = mxfp4, 3 = mxfp8*/, int BLOCK, int U>
 __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restrict__ x, int64_t nchunks,
                                                               uint8_t* __restrict__ codes,
                                                               uint8_t* __restrict__ scales) {
@@ -52,6 +54,19 @@ __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restric
                 const uint32_t packed = e2m1x8_encode_hw(q);
                 if (c < nchunks) {
                     reinterpret_cast<uint32_t*>(codes)[c] = packed;
+                    if ((lane % L) == 0) scales[c / L] = (uint8_t)(e + 127);
+                }
+            } else if (FMT == 3) {
+                // MXFP8: values above 448 saturate (cvt ... satfinite)
+                const int e = mx8_exponent(amax_b);
+                const float inv = exp2_int(-e);  // x * 2**-e == x / 2**e exactly
+                uint2 w;
+                w.x = e4m3x2_encode_hw(v[u][0] * inv, v[u][1] * inv) |
+                      (e4m3x2_encode_hw(v[u][2] * inv, v[u][3] * inv) << 16);
+                w.y = e4m3x2_encode_hw(v[u][4] * inv, v[u][5] * inv) |
+                      (e4m3x2_encode_hw(v[u][6] * inv, v[u][7] * inv) << 16);
+                if (c < nchunks) {
+                    reinterpret_cast<uint2*>(codes)[c] = w;
                     if ((lane % L) == 0) scales[c / L] = (uint8_t)(e + 127);
                 }
             } else {
@@ -212,6 +227,50 @@ BSQ_API bsq_status bsq_dequantize_mxfp4(const uint8_t* packed, const uint8_t* sc
                                                            nitems, (float*)y);
     }
     return check_launch("bsq_dequantize_mxfp4");
+}
+
+BSQ_API bsq_status bsq_quantize_mxfp8(const void* x, bsq_dtype xt, int64_t rows, int64_t K, uint8_t* codes_e4m3,
+                                      uint8_t* scales_e8m0, bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(xt));
+    BSQ_TRY(check_matrix("bsq_quantize_mxfp8", x, rows, K, 32));
+    if (rows * K == 0) return BSQ_OK;
+    if (!codes_e4m3 || !scales_e8m0) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_mxfp8: null output");
+    if (!aligned(x, 16) || !aligned(codes_e4m3, 8))
+        return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_mxfp8: misaligned pointer");
+    const int64_t nchunks = rows * K / 8;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (xt == BSQ_BF16)
+        launch_fit<flat_quant_kernel<uint16_t, 3, 32, 4>>(nchunks, 4, st, (const uint16_t*)x, nchunks, codes_e4m3,
+                                                            scales_e8m0);
+    else
+        launch_fit<flat_quant_kernel<float, 3, 32, 4>>(nchunks, 4, st, (const float*)x, nchunks, codes_e4m3,
+                                                         scales_e8m0);
+    return check_launch("bsq_quantize_mxfp8");
+}
+
+// MXFP8 dequantize is the e4m3 * 2**(scale - 127) decode of the FP8 stored
+// form with 32-element blocks.
+BSQ_API bsq_status bsq_dequantize_mxfp8(const uint8_t* codes_e4m3, const uint8_t* scales_e8m0, int64_t rows,
+                                        int64_t K, void* y, bsq_dtype yt, bsq_stream_t stream) {
+    BSQ_TRY(check_dtype(yt));
+    BSQ_TRY(check_matrix("bsq_dequantize_mxfp8", codes_e4m3, rows, K, 32));
+    if (rows * K == 0) return BSQ_OK;
+    if (!scales_e8m0 || !y) return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_mxfp8: null pointer");
+    if (!aligned(codes_e4m3, 8) || !aligned(y, 16))
+        return fail(BSQ_ERR_INVALID_ARG, "bsq_dequantize_mxfp8: misaligned pointer");
+    cudaStream_t st = (cudaStream_t)stream;
+    const FastDiv none = make_fastdiv(1);
+    const float* nog = nullptr;
+    if (yt == BSQ_BF16) {
+        const int64_t nb = rows * K / 8;
+        launch_fit<dequant_kernel<FMT_FP8, uint16_t, 32, 4>>(nb, 4, st, codes_e4m3, scales_e8m0, nog, none, nb,
+                                                               (uint16_t*)y);
+    } else {
+        const int64_t nf = rows * K / 4;
+        launch_fit<dequant_kernel<FMT_FP8, float, 32, 4>>(nf, 4, st, codes_e4m3, scales_e8m0, nog, none, nf,
+                                                            (float*)y);
+    }
+    return check_launch("bsq_dequantize_mxfp8");
 }
 
 BSQ_API bsq_status bsq_quantize_fp8(const void* x, bsq_dtype xt, int64_t rows, int64_t K, int block,

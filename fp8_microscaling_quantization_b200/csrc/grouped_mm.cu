@@ -24,15 +24,18 @@
 //               (bf16x2 multiply), swizzled 16-byte shared stores
 //   warp 20     B producer: TMA loads of 64-token x 64-k activation boxes
 //   warp 21     tensor-memory allocation and the single MMA-issuing thread
-// Tile = 128 features x up to 256 tokens, k-step 64; a ring of 4 stages,
-// each a 16 KiB dequantized-weight slot and a 32 KiB activation slot with one
-// full and one empty barrier, so the MMA thread waits once and commits once
-// per k-step (its per-k-step instruction time, not the tensor core, sets the
-// pace of a pipelined loop);
-// two 256-column fp32 accumulators in tensor memory so the epilogue of one
-// tile overlaps the main loop of the next.  Tiles are numbered (expert token
+// By default two CTAs of a cluster work as a pair (cta_group::2) on tiles of
+// 256 features x up to 512 tokens: each CTA dequantizes its 128 features and
+// holds half of the tokens, and every k-step issues two M = 256, N <= 256
+// MMAs on the same dequantized weights.  Single CTAs (output widths that are
+// not a multiple of 256) take 128 x 256 tiles with two accumulators, so one
+// tile's epilogue overlaps the next tile's loop.  k-step 64; a ring of 4
+// stages, each a 16 KiB dequantized-weight slot and a 32 KiB activation slot
+// with one full and one empty barrier, so the MMA thread waits once and
+// commits once per k-step (its per-k-step instruction time, not the tensor
+// core, sets the pace of a pipelined loop).  Tiles are numbered (expert token
 // tile, feature tile) with the feature tile fastest, dealt round-robin to the
-// CTAs; every CTA derives the tile table from offs on the device.
+// CTA groups; every CTA derives the tile table from offs on the device.
 //
 // Forward: A = 128 weight rows x 64 k (K-major).  Backward: A = W^T, 128 k
 // columns x 64 weight rows of the contraction (MN-major); NVFP4's row scale
@@ -59,7 +62,7 @@ using namespace sm100;
 namespace gmm {
 
 constexpr int WM = 128;   // features per CTA (the CTA's share of MMA M)
-constexpr int TN = 256;   // tokens per tile at most (MMA N)
+constexpr int TN = 256;   // tokens per MMA at most (MMA N)
 constexpr int BK = 64;
 constexpr int XBOX = 64;  // token rows per TMA box
 // Weights each producer thread converts per k-step (a "unit": 16 or 32
@@ -83,15 +86,27 @@ constexpr int kPrefetch = 4;  // k-steps of packed weights in flight per produce
 
 // Shared-memory plan of a CTA group of CG CTAs (1, or a pair with
 // cta_group::2): a ring of stages, each the dequantized weight slot of one
-// k-step followed by its activation slot (each CTA of a pair holds half of
-// the tile's tokens).  One "full" barrier per stage collects the producer
-// warps' arrivals and the activation bytes, one "empty" barrier receives the
-// MMA commit: the MMA thread waits once and commits once per k-step.
+// k-step followed by its activation slot.  One "full" barrier per stage
+// collects the producer warps' arrivals and the activation bytes, one "empty"
+// barrier receives the MMA commit: the MMA thread waits once and commits once
+// per k-step.
+//
+// A single CTA's tile is 128 features x up to 256 tokens, with two 256-column
+// accumulators so the epilogue of one tile overlaps the next tile's loop.  A
+// pair's tile is 256 features x up to 512 tokens: every k-step issues two
+// M = 256, N <= 256 MMAs (tokens 0-255 and 256-511 of the tile) on the same
+// dequantized weights, which halves the dequantization per tensor-core FLOP
+// for experts with more than 256 tokens; the two MMAs fill the 512 columns of
+// tensor memory, so the pair has one accumulator.  Each CTA of a pair holds
+// its half of both MMAs' tokens: 2 x 128 rows per stage.
 template <int CG>
 struct Plan {
-    static constexpr int STAGES = (CG == 1) ? 4 : 6;
-    static constexpr uint32_t kXStage = (TN / CG) * BK * 2;  // 32 KiB or 16 KiB
-    static constexpr uint32_t kStage = kWStage + kXStage;    // 48 KiB or 32 KiB
+    static constexpr int STAGES = 4;
+    static constexpr int TT = TN * CG;                       // tokens per tile
+    static constexpr int NACC = (CG == 1) ? 2 : 1;           // accumulator buffers
+    static constexpr uint32_t kXHalf = (TN / CG) * BK * 2;   // one MMA's share of a CTA: 32 or 16 KiB
+    static constexpr uint32_t kXStage = kXHalf * CG;         // 32 KiB
+    static constexpr uint32_t kStage = kWStage + kXStage;    // 48 KiB
     static constexpr size_t kBarOffset = (size_t)STAGES * kStage;
     static constexpr int kNumBars = 2 * STAGES + 5;
     static constexpr size_t kSmemBytes = 1024 /* alignment slack */ + kBarOffset + kNumBars * 8 +
@@ -111,7 +126,7 @@ struct Args {
 struct Tile {
     int e;      // expert
     int tok0;   // first token row
-    int ntok;   // tokens in the tile (1..256)
+    int ntok;   // tokens in the tile (1..256 for one CTA, 1..512 for a pair)
     int f0;     // first feature (output column) of the tile
 };
 
@@ -174,10 +189,11 @@ __device__ __forceinline__ Tile decode_tile(int t, int f_tiles, int E, const Sha
         if (sh.tt_prefix[mid] <= tg) lo = mid;
         else hi = mid - 1;
     }
+    constexpr int TT = Plan<CG>::TT;
     Tile ti;
     ti.e = lo;
-    ti.tok0 = sh.seg[lo] + (tg - sh.tt_prefix[lo]) * TN;
-    ti.ntok = min(TN, sh.seg[lo + 1] - ti.tok0);
+    ti.tok0 = sh.seg[lo] + (tg - sh.tt_prefix[lo]) * TT;
+    ti.ntok = min(TT, sh.seg[lo + 1] - ti.tok0);
     ti.f0 = ft * WM * CG;
     return ti;
 }
@@ -369,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
             if (o < prev || o > args.T) bad = 1;
             sh.seg[e] = prev;
             sh.tt_prefix[e] = total;
-            if (!bad) total += (o - prev + TN - 1) / TN;
+            if (!bad) total += (o - prev + P::TT - 1) / P::TT;
             prev = o;
         }
         sh.seg[E] = bad ? 0 : prev;
@@ -412,8 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
         int tile_iter = 0;
         for (int t = group; t < num_tiles; t += ngroups, ++tile_iter) {
             const Tile ti = decode_tile<CG>(t, f_tiles, E, sh);
-            const int acc = tile_iter & 1;
-            if (!wait_bar(&sh.acc_full[acc], (tile_iter >> 1) & 1, sh, args.err)) break;
+            const int acc = tile_iter % P::NACC;
+            if (!wait_bar(&sh.acc_full[acc], (tile_iter / P::NACC) & 1, sh, args.err)) break;
             tc_fence_after();
             const int f = ti.f0 + WM * (int)rank + q * 32 + lane;
             float gf = 1.0f;
@@ -423,6 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
 #pragma unroll 1
             for (int c = 0; c < chunks; ++c) {
                 uint32_t r[16];
+                // token j of the tile is accumulator column j (a pair's second
+                // MMA writes columns 256..511)
                 tmem_ld_32x32b_x16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * TN + c * 16), r);
                 tmem_ld_wait();
                 const int nv = min(16, ti.ntok - c * 16);
@@ -506,9 +524,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
             bool ok = true;
             for (int t = group; t < num_tiles && ok; t += ngroups) {
                 const Tile ti = decode_tile<CG>(t, f_tiles, E, sh);
-                const int n_mma = (ti.ntok + 15) & ~15;
-                const int half = n_mma / CG;  // this CTA's share of the tokens
-                const int nbox = (half + XBOX - 1) / XBOX;
+                // tokens of the tile's first and second MMA, rounded up to 16,
+                // and this CTA's share (rows) of each
+                const int n0 = (min(ti.ntok, TN) + 15) & ~15;
+                const int n1 = (CG == 2 && ti.ntok > TN) ? ((ti.ntok - TN + 15) & ~15) : 0;
+                const int h0 = n0 / CG, h1 = n1 / CG;
+                const int nbox0 = (h0 + XBOX - 1) / XBOX, nbox1 = (h1 + XBOX - 1) / XBOX;
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
                     const int s = it % P::STAGES;
                     if (!wait_bar(&sh.empty[s], ((it / P::STAGES) & 1) ^ 1, sh, args.err)) {
@@ -517,16 +538,21 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                     }
                     uint8_t* dst = sh.stage + s * P::kStage + kWStage;
                     if (CG == 1) {
+                        const int nbox = nbox0;
                         mbar_arrive_expect_tx(&sh.full[s], nbox * kXBoxBytes);
                         for (int b = 0; b < nbox; ++b)
                             tma_load_2d(dst + b * kXBoxBytes, &tmap_x, &sh.full[s], ks * BK, ti.tok0 + b * XBOX);
                     } else {
-                        // both CTAs' boxes complete on the leader's barrier
-                        if (leader) mbar_arrive_expect_tx(&sh.full[s], 2 * nbox * kXBoxBytes);
+                        // both CTAs' boxes complete on the leader's barrier; the
+                        // second MMA's rows go kXHalf into the slot
+                        if (leader) mbar_arrive_expect_tx(&sh.full[s], 2 * (nbox0 + nbox1) * kXBoxBytes);
                         const uint32_t bar = mapa_shared(smem_u32(&sh.full[s]), 0);
-                        for (int b = 0; b < nbox; ++b)
+                        for (int b = 0; b < nbox0; ++b)
                             tma_load_2d_pair(dst + b * kXBoxBytes, &tmap_x, bar, ks * BK,
-                                             ti.tok0 + (int)rank * half + b * XBOX);
+                                             ti.tok0 + (int)rank * h0 + b * XBOX);
+                        for (int b = 0; b < nbox1; ++b)
+                            tma_load_2d_pair(dst + P::kXHalf + b * kXBoxBytes, &tmap_x, bar, ks * BK,
+                                             ti.tok0 + TN + (int)rank * h1 + b * XBOX);
                     }
                 }
             }
@@ -551,10 +577,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
             bool ok = true;
             for (int t = group; t < num_tiles && ok; t += ngroups, ++tile_iter) {
                 const Tile ti = decode_tile<CG>(t, f_tiles, E, sh);
-                const uint32_t n_mma = (uint32_t)((ti.ntok + 15) & ~15);
-                const uint32_t idesc = idesc_bf16_ab(WM * CG, n_mma, DIR == BSQ_BWD ? 1u : 0u, 0u);
-                const int acc = tile_iter & 1;
-                if (!wait_bar(&sh.acc_empty[acc], ((tile_iter >> 1) & 1) ^ 1, sh, args.err)) break;
+                const uint32_t n0 = (uint32_t)((min(ti.ntok, TN) + 15) & ~15);
+                const uint32_t n1 = (CG == 2 && ti.ntok > TN) ? (uint32_t)((ti.ntok - TN + 15) & ~15) : 0u;
+                const uint32_t idesc0 = idesc_bf16_ab(WM * CG, n0, DIR == BSQ_BWD ? 1u : 0u, 0u);
+                const uint32_t idesc1 = idesc_bf16_ab(WM * CG, n1 ? n1 : 16u, DIR == BSQ_BWD ? 1u : 0u, 0u);
+                const int acc = tile_iter % P::NACC;
+                if (!wait_bar(&sh.acc_empty[acc], ((tile_iter / P::NACC) & 1) ^ 1, sh, args.err)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * TN);
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
@@ -572,8 +600,13 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                         // the start address field (bits 0-13) cannot carry: the
                         // stage lies below 256 KiB of shared memory
                         const uint64_t ad = ad0 + kAStep * k16, bd = bd0 + kBStep * k16;
-                        if (CG == 1) mma_bf16_ss(d_tmem, ad, bd, idesc, (ks | k16) != 0 ? 1u : 0u);
-                        else mma_bf16_ss_pair(d_tmem, ad, bd, idesc, (ks | k16) != 0 ? 1u : 0u);
+                        const uint32_t accum = (ks | k16) != 0 ? 1u : 0u;
+                        if (CG == 1) {
+                            mma_bf16_ss(d_tmem, ad, bd, idesc0, accum);
+                        } else {
+                            mma_bf16_ss_pair(d_tmem, ad, bd, idesc0, accum);
+                            if (n1) mma_bf16_ss_pair(d_tmem + TN, ad, bd + (P::kXHalf >> 4), idesc1, accum);
+                        }
                     }
                     if (CG == 1) mma_commit(&sh.empty[s]);
                     else mma_commit_pair_multicast(&sh.empty[s], 0x3);
@@ -724,14 +757,16 @@ BSQ_API bsq_status bsq_grouped_mm_fp4(bsq_format fmt, bsq_dir dir, const void* a
     args.T = (int)T;
     args.N = (int)N;
     args.K = (int)K;
-    // Single CTAs by default.  The environment variable BSQ_GMM_CTA_PAIR=1
-    // selects CTA pairs (M = 256 features per tile, cta_group::2) where the
-    // output width allows it; both measured within a few per cent of each
-    // other with 16-weight producer units.
+    // CTA pairs (256 features x 512 tokens per tile, cta_group::2) wherever
+    // the output width is a multiple of 256: they dequantize each weight tile
+    // once for twice the tokens and measured 15-25% faster than single CTAs.
+    // The environment variable BSQ_GMM_CTA_PAIR=0 selects single CTAs.
     const char* pair_env = getenv("BSQ_GMM_CTA_PAIR");
-    const int cg = (pair_env && pair_env[0] == '1' && out_w % (2 * gmm::WM) == 0) ? 2 : 1;
+    const bool pairs_off = pair_env && pair_env[0] == '0';
+    const int cg = (!pairs_off && out_w % (2 * gmm::WM) == 0) ? 2 : 1;
     const int64_t f_tiles = out_w / (gmm::WM * cg);
-    const int64_t max_groups = ((T + gmm::TN - 1) / gmm::TN + E) * f_tiles;
+    const int64_t tile_tok = (int64_t)gmm::TN * cg;
+    const int64_t max_groups = ((T + tile_tok - 1) / tile_tok + E) * f_tiles;
     cudaStream_t s = (cudaStream_t)stream;
     if (cg == 2) {
         if (fmt == BSQ_MXFP4)

@@ -49,7 +49,7 @@ typedef enum {
 } bsq_status;
 
 typedef enum { BSQ_BF16 = 0, BSQ_FP32 = 1 } bsq_dtype;
-typedef enum { BSQ_FP8 = 0, BSQ_MXFP4 = 1, BSQ_NVFP4 = 2 } bsq_format;
+typedef enum { BSQ_FP8 = 0, BSQ_MXFP4 = 1, BSQ_NVFP4 = 2, BSQ_MXFP8 = 3 } bsq_format;
 typedef enum { BSQ_FWD = 0, BSQ_BWD = 1 } bsq_dir;
 
 /* Bits of the device error word written by bsq_grouped_mm_fp4. */
@@ -118,6 +118,42 @@ bsq_status bsq_dequantize_nvfp4(const uint8_t* packed, const uint8_t* scales_e4m
                                 const float* row_scale, int64_t rows, int64_t K, void* y,
                                 bsq_dtype yt, bsq_stream_t stream);
 
+/* ----------------------------------------------- paged NVFP4 KV cache ---
+ * NeMo AutoModel model-filter page, dequantize_kv_cache: a list of nblocks
+ * quantized blocks, block b holding block_tokens * heads rows of 128 values
+ * (row = token-in-block * heads + head):
+ *   values[b]  e2m1 codes [rows, 64] (two per byte, even column low nibble)
+ *   scales[b]  e4m3 scales [rows, 8] (row-major; the pages' swizzled
+ *              from_blocked layout is not defined there)
+ *   amax[b]    one fp32; the block's global scale is amax / (6 * 448)
+ * Output y [1, nblocks * block_tokens, heads, 128] (bf16 or fp32, 16-byte
+ * aligned): token t of block b is token b * block_tokens + t, each value
+ * (e2m1 * e4m3) * g in binary32 with one final rounding to yt.
+ * values, scales and amax are device arrays of nblocks device pointers
+ * (8-byte aligned arrays; the pointed-to blocks may have any alignment).
+ * One launch for all blocks; at most 2**32 output items (8 bf16 or 4 fp32). */
+bsq_status bsq_dequantize_kv_cache_nvfp4(const uint8_t* const* values, const uint8_t* const* scales,
+                                         const float* const* amax, int64_t nblocks, int64_t block_tokens,
+                                         int64_t heads, void* y, bsq_dtype yt, bsq_stream_t stream);
+
+/* ------------------------------------------- static two-level NVFP4 -----
+ * ModelOpt tensor_quantizer page, StaticBlockScaleQuantizer (two-level
+ * scaling with an FP8-quantized block scale): fake-quant of x [rows, K]
+ * (K % 16 == 0) with a calibrated amax per 16-element block and a global amax A:
+ *   pts = A / 6 (1e-8 where A / 6 <= 1e-8),  min_value = (2**-9 / 448) * pts,
+ *   sb  = amax_b / 6 (min_value where amax_b / 6 <= min_value),
+ *   sq  = e4m3(sb * 448 / pts) / (448 / pts),   y = e2m1(x / sq) * sq,
+ * binary32 with one rounding per operation in this order, one final rounding
+ * to t.  The pages do not print scaled_e4m3: the 448 / pts map and its
+ * inverse as a division by the same factor are this library's reading.
+ *   x, y [rows, K] bf16 or fp32 (t), 16-byte aligned; y == x (in place) is
+ *   allowed, any other overlap is rejected.  block_amax [rows, K/16] fp32 and
+ *   global_amax (one fp32) are device pointers.  The straight-through
+ *   backward is the identity: use the gradient as is. */
+bsq_status bsq_fake_quantize_nvfp4_static(const void* x, bsq_dtype t, int64_t rows, int64_t K,
+                                          const float* block_amax, const float* global_amax, void* y,
+                                          bsq_stream_t stream);
+
 /* ---------------------------------------------------------------- MXFP4 --
  * mxfp4 page, quantize_mxfp4: K % 32 == 0; per 32-block scale
  * 2**(floor(log2(amax)) - 2) (exact floor; an all-zero block takes 2**-127;
@@ -131,6 +167,24 @@ bsq_status bsq_quantize_mxfp4(const void* x, bsq_dtype xt, int64_t rows, int64_t
 /* mxfp4 page, dequantize_mxfp4: y = e2m1 * 2**(scale byte - 127) (exact;
  * scale byte 0xFF is NaN). */
 bsq_status bsq_dequantize_mxfp4(const uint8_t* packed, const uint8_t* scales_e8m0, int64_t rows,
+                                int64_t K, void* y, bsq_dtype yt, bsq_stream_t stream);
+
+/* ---------------------------------------------------------------- MXFP8 --
+ * ModelOpt tensor_quantizer page, is_mxfp(8) / _real_quantize: e4m3 elements
+ * with one e8m0 scale per 32-column block.  The pages do not print the
+ * quantize body; the scale carries the mxfp4 page's rule over to e4m3's
+ * largest exponent: 2**(floor(log2(amax)) - 8) (exact floor; an all-zero block
+ * takes 2**-127; exponent clamped to [-127, 127]), stored as exponent + 127;
+ * code = e4m3 round-to-nearest-even of w / scale, saturating at +-448 (the
+ * block maximum lands in [256, 512) before rounding).  K % 32 == 0.
+ *   x [rows, K] bf16 or fp32 (16-byte aligned); codes_e4m3 [rows, K] uint8
+ *   (8-byte aligned); scales_e8m0 [rows, K/32]. */
+bsq_status bsq_quantize_mxfp8(const void* x, bsq_dtype xt, int64_t rows, int64_t K,
+                              uint8_t* codes_e4m3, uint8_t* scales_e8m0, bsq_stream_t stream);
+
+/* y = e4m3 * 2**(scale byte - 127) (exact in fp32; scale byte 0xFF and codes
+ * 0x7F / 0xFF are NaN).  y [rows, K] bf16 or fp32 (16-byte aligned). */
+bsq_status bsq_dequantize_mxfp8(const uint8_t* codes_e4m3, const uint8_t* scales_e8m0, int64_t rows,
                                 int64_t K, void* y, bsq_dtype yt, bsq_stream_t stream);
 
 /* ------------------------------------------------------------------ FP8 --

@@ -101,11 +101,11 @@ def test_gemm_edge_offsets(B, oracle, fmt):
 
 
 @pytest.mark.parametrize("fmt", [1, 2])
-def test_gemm_cta_pairs(B, oracle, fmt, monkeypatch):
-    # BSQ_GMM_CTA_PAIR=1 runs 256-feature tiles on CTA pairs (cta_group::2);
-    # an output width of 384 is not a multiple of 256 and falls back to single
-    # CTAs within the same call sequence
-    monkeypatch.setenv("BSQ_GMM_CTA_PAIR", "1")
+def test_gemm_single_ctas(B, oracle, fmt, monkeypatch):
+    # BSQ_GMM_CTA_PAIR=0 runs 128-feature x 256-token tiles on single CTAs
+    # instead of the default CTA pairs (256 features x 512 tokens,
+    # cta_group::2); the same shapes as the default-mode tests
+    monkeypatch.setenv("BSQ_GMM_CTA_PAIR", "0")
     full_check(B, oracle, fmt, T=300, K=256, N=256, E=4, seed=11)
     full_check(B, oracle, fmt, T=2048, K=1024, N=512, E=8, seed=12)
     full_check(B, oracle, fmt, T=400, K=256, N=256, E=6, seed=14, offs=[0, 1, 130, 130, 390, 390])
@@ -114,7 +114,8 @@ def test_gemm_cta_pairs(B, oracle, fmt, monkeypatch):
 
 @pytest.mark.parametrize("fmt", [1, 2])
 def test_gemm_output_width_not_256(B, oracle, fmt):
-    # output width a multiple of 128 but not of 256, K not a multiple of 128
+    # output width a multiple of 128 but not of 256 (single CTAs even in the
+    # default mode), K not a multiple of 128
     full_check(B, oracle, fmt, T=300, K=384, N=384, E=3, seed=17)
 
 
@@ -137,12 +138,15 @@ def test_gemm_rejects_bad_shapes(B):
         B.bsq_grouped_mm_fp4(B.Format.FP8, B.Direction.FWD, x, p, s, None, offs)
 
 
+@pytest.mark.parametrize("pair", ["0", "1"])
 @pytest.mark.parametrize("fmt", [1, 2])
-def test_gemm_full_size_sampled(B, oracle, fmt):
+def test_gemm_full_size_sampled(B, oracle, fmt, pair, monkeypatch):
     """T=16384, K=7168, N=2048, E=32 with Zipf(1.1) routing (one empty expert):
     all rows of the two smallest non-empty experts, the first and last row of
-    every expert and 12 seeded rows per expert, forward and backward."""
+    every expert and 12 seeded rows per expert, forward and backward; single
+    CTAs (256-token tiles) and CTA pairs (512-token tiles)."""
     from fp8_microscaling_quantization_b200 import synth
+    monkeypatch.setenv("BSQ_GMM_CTA_PAIR", pair)
     prob = synth.moe_problem()
     x, w, go, offs = prob["x"], prob["w"], prob["grad_out"], prob["offs"]
     packed, scales, g = quantize_weights(oracle, fmt, w)
@@ -167,4 +171,4 @@ def test_gemm_full_size_sampled(B, oracle, fmt):
         assert err == 0
         ref = oracle.grouped_mm_rows(fmt, backward, a, packed, scales, g, offs, rows)
         check_rows(got[rows], ref, a, Wmax, 2048 if backward else 7168,
-                   f"full-size fmt={fmt} {'bwd' if backward else 'fwd'}")
+                   f"full-size fmt={fmt} pair={pair} {'bwd' if backward else 'fwd'}")

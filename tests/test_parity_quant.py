@@ -231,6 +231,72 @@ def test_mxfp4_dequant_all_scale_codes(B, oracle):
         assert_bits_equal(got, want, f"dequant {dt}")
 
 
+# ---------------------------------------------------------------- MXFP8 -----
+
+def test_mxfp8_full_size_expert_weights(B, S, oracle):
+    """[8, 2048, 7168] routed-expert weights as MXFP8: scales, codes and both
+    dequantized outputs compared in full."""
+    x = S.expert_weights()
+    c, s = B.bsq_quantize_mxfp8(dev_bf16(x))
+    yb = B.bsq_dequantize_mxfp8(c, s)
+    yf = B.bsq_dequantize_mxfp8(c, s, out_dtype=B.DType.FP32)
+    oc, os_ = oracle.quantize_mxfp8(x)
+    del x
+    assert_bits_equal(host_bits(s), os_, "e8m0 scales")
+    assert_bits_equal(host_bits(c), oc, "e4m3 codes")
+    assert_bits_equal(host_bits(yb), oracle.dequantize_mxfp8(oc, os_), "dequant bf16")
+    assert_bits_equal(host_bits(yf), oracle.dequantize_mxfp8(oc, os_, out_dtype=oracle.F32), "dequant fp32")
+    assert (host_bits(s) == 0).sum() == 8 * 16  # the exact-zero blocks
+
+
+@pytest.mark.parametrize("rows,K", [(3, 32), (77, 96), (1000, 1024)])
+def test_mxfp8_small_and_ragged(B, S, oracle, rows, K):
+    x = S.nvfp4_matrix(rows=rows, cols=K, seed=rows * 11 + K)
+    c, s = B.bsq_quantize_mxfp8(dev_bf16(x))
+    oc, os_ = oracle.quantize_mxfp8(x)
+    assert_bits_equal(host_bits(s), os_, "scales")
+    assert_bits_equal(host_bits(c), oc, "codes")
+    # fp32 input far below 2**-118: the block exponent sits on the e8m0 floor
+    xf = f32_of(x) * np.float32(1e-36)
+    c, s = B.bsq_quantize_mxfp8(dev(xf))
+    oc, os_ = oracle.quantize_mxfp8(xf)
+    assert (os_ == 0).any()
+    assert_bits_equal(host_bits(s), os_, "scales fp32 tiny")
+    assert_bits_equal(host_bits(c), oc, "codes fp32 tiny")
+
+
+def test_mxfp8_every_bf16_value_as_quotient(B, oracle):
+    """Blocks led by 256 have exponent 0, so the e4m3 rounding sees every bf16
+    value of magnitude below 512 unchanged: ties, subnormals, signed zeros and
+    the saturation of (448, 512)."""
+    vals = edge_bf16_values()
+    v = vals[np.abs(f32_of(vals)) < 512]
+    n = -(-v.size // 31)
+    flat = np.zeros(n * 31, np.uint16)
+    flat[:v.size] = v
+    blocks = np.zeros((n, 32), np.uint16)
+    blocks[:, 0] = 0x4380  # 256
+    blocks[:, 1:] = flat.reshape(n, 31)
+    c, s = B.bsq_quantize_mxfp8(dev_bf16(blocks))
+    oc, os_ = oracle.quantize_mxfp8(blocks)
+    assert np.all(os_ == 127)
+    assert_bits_equal(host_bits(s), os_, "scales")
+    assert_bits_equal(host_bits(c), oc, "codes")
+
+
+def test_mxfp8_dequant_all_scale_codes(B, oracle):
+    rng = np.random.default_rng(14)
+    codes = rng.integers(0, 256, (256, 32), dtype=np.uint8)  # includes the NaN codes
+    scales = np.arange(256, dtype=np.uint8).reshape(256, 1)  # 255 = NaN
+    for dt, odt in ((B.DType.BF16, oracle.BF16), (B.DType.FP32, oracle.F32)):
+        y = B.bsq_dequantize_mxfp8(dev(codes), dev(scales), out_dtype=dt)
+        want = oracle.dequantize_mxfp8(codes, scales, out_dtype=odt)
+        got = host_bits(y)
+        nan = np.isnan(f32_of(want) if odt == oracle.BF16 else want)
+        assert np.array_equal(np.isnan(f32_of(got) if odt == oracle.BF16 else got.view(np.float32)), nan)
+        assert_bits_equal(got[~nan], want[~nan], f"dequant {dt}")
+
+
 # ------------------------------------------------------------------ FP8 -----
 
 @pytest.mark.parametrize("block", [16, 32])
