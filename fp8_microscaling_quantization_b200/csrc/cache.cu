@@ -14,6 +14,9 @@
 namespace bsq {
 
 // ------------------------------------------------------- quantize_cache ----
+template <int FMT, int L>
+__device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg, float out[8]);
+
 // S lanes per row (S a power of two, 2 <= S <= 32; 32/S rows per warp); lane
 // i of a row walks the chunks i, i + S, ...  of the zero-padded row, so the
 // L lanes of a block are adjacent.  VEC: rows are 16-byte aligned and C % 8 == 0.
@@ -34,7 +37,7 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
         const bool row_ok = r < rows;
         const T* xr = x + (row_ok ? r : 0) * C;
         T* yr = y + (row_ok ? r : 0) * C;
-        float g = 0.0f;
+        float g = 0.0f, rg = 0.0f;
         if (FMT == BSQ_NVFP4) {
             float m = 0.0f;
             for (int64_t c0 = 0; c0 < cpr; c0 += S) {
@@ -49,6 +52,7 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
             }
             m = group_max<S>(m);
             g = __fdiv_rn(m, kNvGlobalDiv);
+            rg = nv_recip_or_zero(g);
         }
         for (int64_t c0 = 0; c0 < cpr; c0 += S) {
             const int64_t c = c0 + sl;
@@ -61,38 +65,8 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
 #pragma unroll
                 for (int j = 0; j < 8; ++j) v[j] = 0.0f;
             }
-            const float amax_b = group_max<L>(amax8(v));
             float out[8];
-            if (FMT == BSQ_FP8) {
-                const float p = pow2_scale(amax_b, kE4M3Max);
-                const float inv = exp2_int(127 - f32_biased_exp(p));
-#pragma unroll
-                for (int j = 0; j < 8; j += 2) {
-                    const float2 d = e4m3x2_decode_hw(e4m3x2_encode_hw(v[j] * inv, v[j + 1] * inv));
-                    out[j] = d.x * p;
-                    out[j + 1] = d.y * p;
-                }
-            } else if (FMT == BSQ_MXFP4) {
-                const float p = pow2_scale(amax_b, kE2M1Max);
-                const float inv = exp2_int(127 - f32_biased_exp(p));
-                float q[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) q[j] = v[j] * inv;
-                const uint32_t pk = e2m1x8_encode_hw(q);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) out[j] = e2m1_decode((pk >> (4 * j)) & 15u) * p;
-            } else {
-                if (g == 0.0f) {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) out[j] = 0.0f;
-                } else {
-                    const float s = e4m3_decode(nv_scale_byte(amax_b, g));
-                    const float d = __fmul_rn(s, g);
-                    const uint32_t pk = e2m1x8_of_quotient(v, d);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(__fmul_rn(e2m1_decode((pk >> (4 * j)) & 15u), s), g);
-                }
-            }
+            cache_chunk<FMT, L>(v, g, rg, out);
             if (row_ok && c < cpr && n > 0) {
                 if (VEC && n >= 8) store8(yr + c * 8, out);
                 else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
@@ -118,12 +92,13 @@ __device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg,
     } else if (FMT == BSQ_MXFP4) {
         const float p = pow2_scale(amax_b, kE2M1Max);
         const float inv = exp2_int(127 - f32_biased_exp(p));
-        float q[8];
+        float q[8], e[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) q[j] = v[j] * inv;
-        const uint32_t pk = e2m1x8_encode_hw(q);
+        e2m1x8_decode_hw(e2m1x8_encode_hw(q), e);
+        // e * p is exact; adding +0 turns code 8's -0 into the table's +0
 #pragma unroll
-        for (int j = 0; j < 8; ++j) out[j] = e2m1_decode((pk >> (4 * j)) & 15u) * p;
+        for (int j = 0; j < 8; ++j) out[j] = __fmaf_rn(e[j], p, 0.0f);
     } else {
         if (g == 0.0f) {
 #pragma unroll
@@ -131,9 +106,11 @@ __device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg,
         } else {
             const float s = e4m3_decode(nv_scale_code(amax_b, g, rg));
             const float d = __fmul_rn(s, g);
-            const uint32_t pk = e2m1x8_of_quotient(v, d);
+            float e[8];
+            e2m1x8_decode_hw(e2m1x8_of_quotient(v, d), e);
+            // (e2m1 * s) is exact (and +0 for code 8), then one rounding by g
 #pragma unroll
-            for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(__fmul_rn(e2m1_decode((pk >> (4 * j)) & 15u), s), g);
+            for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(__fmaf_rn(e[j], s, 0.0f), g);
         }
     }
 }
@@ -148,21 +125,19 @@ __global__ void __launch_bounds__(kThreads) cache_flat_kernel(const T* __restric
     const int lane = threadIdx.x & 31;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < nchunks; base += U * stride) {
-        float v[U][8];
+        Raw8<T> raw[U];  // every chunk's load in flight before any arithmetic
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t c = base + u * stride + lane;
-            if (c < nchunks) load8(x + c * 8, v[u]);
-            else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
-            }
+            if (c < nchunks) raw[u].load(x + c * 8);
+            else raw[u].zero();
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t c = base + u * stride + lane;
-            float out[8];
-            cache_chunk<FMT, L>(v[u], 0.0f, 0.0f, out);
+            float v[8], out[8];
+            raw[u].get(v);
+            cache_chunk<FMT, L>(v, 0.0f, 0.0f, out);
             if (c < nchunks) store8(y + c * 8, out);
         }
     }

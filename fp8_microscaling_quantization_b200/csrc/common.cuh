@@ -144,9 +144,15 @@ __device__ __forceinline__ void build_e2m1_lut(float2* lut) {
 // are the codes of RN(v / d); only when a bracket straddles a rounding
 // boundary (rare) or d is out of range is the quotient computed by IEEE
 // division.
+__device__ __forceinline__ uint32_t e2m1x8_of_quotient_r(const float v[8], float d, float r);
+
 __device__ __forceinline__ uint32_t e2m1x8_of_quotient(const float v[8], float d) {
+    return e2m1x8_of_quotient_r(v, d, __frcp_rn(d));
+}
+
+// The same with r = RN(1 / d) supplied by the caller (a per-scale table).
+__device__ __forceinline__ uint32_t e2m1x8_of_quotient_r(const float v[8], float d, float r) {
     if (d >= 2.3509887e-38f /* 2**-125 */ && d <= 4.2535296e37f /* 2**125 */) {
-        const float r = __frcp_rn(d);
         float lo[8], hi[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -236,6 +242,30 @@ __device__ __forceinline__ void load16(const float* p, float v[16]) {
         v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
     }
 }
+
+// 8 consecutive elements kept as loaded (bf16: one uint4, fp32: two float4)
+// and widened to binary32 on use: a bf16 chunk in flight costs 4 registers.
+template <typename T> struct Raw8;
+template <> struct Raw8<uint16_t> {
+    uint4 r;
+    __device__ __forceinline__ void load(const uint16_t* p) { r = *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ void zero() { r = make_uint4(0u, 0u, 0u, 0u); }
+    __device__ __forceinline__ void get(float v[8]) const {
+        v[0] = bf16_lo(r.x); v[1] = bf16_hi(r.x); v[2] = bf16_lo(r.y); v[3] = bf16_hi(r.y);
+        v[4] = bf16_lo(r.z); v[5] = bf16_hi(r.z); v[6] = bf16_lo(r.w); v[7] = bf16_hi(r.w);
+    }
+};
+template <> struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p) {
+        a = reinterpret_cast<const float4*>(p)[0];
+        b = reinterpret_cast<const float4*>(p)[1];
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void get(float v[8]) const {
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+};
 
 // Grid of a multiple of the SM count: enough CTAs for `items` at
 // `per_thread` items per thread, capped at 8 CTAs per SM (grid-stride loops).

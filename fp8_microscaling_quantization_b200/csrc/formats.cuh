@@ -116,6 +116,25 @@ __device__ __forceinline__ uint32_t e2m1x8_encode_hw(const float v[8]) {
     return out;
 }
 
+// Four bytes of packed e2m1 codes -> eight binary32 values (code 2i + j from
+// nibble j of byte i), by the hardware conversion to f16x2 and f16 -> f32
+// (both exact).  Code 8 gives -0.0 here; a caller that needs the table's
+// +0.0 adds +0.0 (fma(v, s, 0.0f) rounds v * s once and turns -0 into +0).
+__device__ __forceinline__ void e2m1x8_decode_hw(uint32_t w, float v[8]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t h2;
+        asm("{\n\t.reg .b8 t;\n\t"
+            "cvt.u8.u32 t, %1;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+            : "=r"(h2)
+            : "r"(w >> (8 * i)));
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
 // e2m1 code -> binary32.  Magnitude m: 0 and 1 are 0 and 0.5; m >= 2 is
 // (1 + (m & 1) / 2) * 2**((m >> 1) - 1).  Code 8 decodes to +0.0.
 __device__ __forceinline__ float e2m1_decode(uint32_t c) {

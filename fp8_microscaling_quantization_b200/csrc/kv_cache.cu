@@ -10,10 +10,12 @@
 // (b + 1) * block_tokens), so the output of block b is one contiguous range.
 //
 // One fused launch for every block: an item is 8 outputs (bf16, one 16-byte
-// store) or 4 (fp32); the block of an item comes from a constant-divisor
-// multiply, and the block's three pointers from small device arrays that stay
-// in L1 / L2.  Codes stream through once; the e2m1 byte table lives in shared
-// memory.
+// store) or 4 (fp32), consecutive lanes take consecutive items, and each warp
+// walks a run of 32 * U items.  The block of an item comes from a
+// constant-divisor multiply; a lane loads the block's pointers and global
+// scale only when its item enters another block, so the load pipe carries
+// little beyond the codes, the scale bytes and the stores.  e2m1 codes are
+// decoded by the hardware e2m1 -> f16x2 conversion.
 #include "common.cuh"
 
 namespace bsq {
@@ -44,39 +46,51 @@ __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const uint8_t* con
                                                               FastDiv items_per_block, int64_t nitems,
                                                               TOUT* __restrict__ y) {
     constexpr int EPI = (sizeof(TOUT) == 2) ? 8 : 4;  // outputs per item
-    __shared__ float2 lut[256];
-    build_e2m1_lut(lut);
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nitems; base += U * stride) {
+    constexpr int RUN = 32 * U;                       // items of one warp's run
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+    // the block's pointers and global scale, reloaded only when a lane's item
+    // moves into another block (a run lies in one block unless it straddles
+    // a boundary)
+    uint32_t cur = 0xFFFFFFFFu;
+    const uint8_t* vb = nullptr;
+    const uint8_t* sb = nullptr;
+    float g = 0.0f;
+    for (int64_t run = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); run * RUN < nitems;
+         run += warps) {
         uint32_t w[U], sc[U];
-        float g[U];
+        float gr[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t it = base + u * stride;
+            const int64_t it = run * RUN + u * 32 + lane;  // consecutive lanes, consecutive items
             w[u] = sc[u] = 0u;
-            g[u] = 0.0f;
+            gr[u] = 0.0f;
             if (it < nitems) {
                 const uint32_t b = fdiv((uint32_t)it, items_per_block);
+                if (b != cur) {
+                    cur = b;
+                    vb = values[b];
+                    sb = scales[b];
+                    g = __fdiv_rn(ld_f32_any(amax[b]), 2688.0f);
+                }
                 const uint32_t o = (uint32_t)it - b * items_per_block.d;  // item within the block
-                w[u] = ld_codes(values[b], o, EPI / 2);
+                w[u] = ld_codes(vb, o, EPI / 2);
                 // element o * EPI of the block: row (o * EPI) / 128, scale column ((o * EPI) % 128) / 16,
                 // i.e. scale byte (o * EPI) / 16 of the row-major [rows, 8] scales
-                sc[u] = scales[b][(o * EPI) >> 4];
-                g[u] = __fdiv_rn(ld_f32_any(amax[b]), 2688.0f);
+                sc[u] = sb[(o * EPI) >> 4];
+                gr[u] = g;
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t it = base + u * stride;
+            const int64_t it = run * RUN + u * 32 + lane;
             if (it >= nitems) continue;
             const float s = e4m3_decode(sc[u]);
-            float v[8];
+            float e[8], v[8];
+            e2m1x8_decode_hw(w[u], e);  // fp32 output: only the first 4 are used
+            // (e2m1 * s) is exact, and +0 for code 8; then one rounding by g
 #pragma unroll
-            for (int i = 0; i < EPI / 2; ++i) {
-                const float2 t = lut[(w[u] >> (8 * i)) & 0xFFu];
-                v[2 * i] = __fmul_rn(__fmul_rn(t.x, s), g[u]);
-                v[2 * i + 1] = __fmul_rn(__fmul_rn(t.y, s), g[u]);
-            }
+            for (int i = 0; i < EPI; ++i) v[i] = __fmul_rn(__fmaf_rn(e[i], s, 0.0f), gr[u]);
             TOUT* dst = y + it * EPI;
             if (sizeof(TOUT) == 2) {
                 uint4 o4;
@@ -114,8 +128,8 @@ BSQ_API bsq_status bsq_dequantize_kv_cache_nvfp4(const uint8_t* const* values, c
     const FastDiv ipb = make_fastdiv((uint32_t)items_per_block);
     cudaStream_t st = (cudaStream_t)stream;
     if (yt == BSQ_BF16)
-        launch_fit<kv_dequant_kernel<uint16_t, 4>>(nitems, 4, st, values, scales, amax, ipb, nitems, (uint16_t*)y);
+        launch_fit<kv_dequant_kernel<uint16_t, 8>>(nitems, 8, st, values, scales, amax, ipb, nitems, (uint16_t*)y);
     else
-        launch_fit<kv_dequant_kernel<float, 4>>(nitems, 4, st, values, scales, amax, ipb, nitems, (float*)y);
+        launch_fit<kv_dequant_kernel<float, 8>>(nitems, 8, st, values, scales, amax, ipb, nitems, (float*)y);
     return check_launch(fn);
 }

@@ -12,8 +12,13 @@
 // binary32 throughout, every product and quotient rounded once, in this order.
 // The straight-through backward is the identity (no kernel).
 //
-// One lane per 16-element block, two blocks in flight per lane; the e2m1
-// codes of x / sq come from the division-free exact quotient rounding.
+// A lane is 8 consecutive elements (one 16-byte load and store), so a warp
+// instruction covers one contiguous span; the two lanes of a block each
+// derive its scale.  Four chunks in flight per lane.  The physical scale of
+// each of the 128 positive e4m3 codes (and its reciprocal) is tabulated per
+// CTA, since f is fixed per launch; the e2m1 codes of x / sq come from the
+// division-free exact quotient rounding, and decode back through the
+// hardware e2m1 -> f16x2 conversion.
 #include "common.cuh"
 
 namespace bsq {
@@ -26,43 +31,51 @@ template <typename T, int U>
 __global__ void __launch_bounds__(kThreads) nv_static_fq_kernel(const T* __restrict__ x,
                                                                 const float* __restrict__ block_amax,
                                                                 const float* __restrict__ global_amax,
-                                                                int64_t nblocks, T* y) {
+                                                                int64_t nchunks, T* y) {
+    // the physical scale of every positive e4m3 code, and its reciprocal, for
+    // this launch's global amax (one division per code, not per block)
+    __shared__ float sq_of[128], rsq_of[128];
     float pts = __fdiv_rn(__ldg(global_amax), 6.0f);
     if (pts <= 1e-8f) pts = 1e-8f;
     const float min_value = __fmul_rn(kStaticMinRatio, pts);
     const float f = __fdiv_rn(448.0f, pts);
+    for (int c = threadIdx.x; c < 128; c += kThreads) {
+        const float sq = __fdiv_rn(e4m3_decode((uint32_t)c), f);
+        sq_of[c] = sq;
+        rsq_of[c] = __frcp_rn(sq);
+    }
+    __syncthreads();
     const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nblocks; base += U * stride) {
-        float v[U][16], a[U];
+    for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nchunks; base += U * stride) {
+        float v[U][8], a[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t b = base + u * stride;
-            if (b < nblocks) {
-                load16(x + b * 16, v[u]);
-                a[u] = __ldg(block_amax + b);
+            const int64_t c = base + u * stride;
+            if (c < nchunks) {
+                load8(x + c * 8, v[u]);
+                a[u] = __ldg(block_amax + (c >> 1));
             } else {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) v[u][j] = 0.0f;
+                for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
                 a[u] = 0.0f;
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t b = base + u * stride;
-            if (b >= nblocks) continue;
+            const int64_t c = base + u * stride;
+            if (c >= nchunks) continue;
+            // both lanes of a block derive the same scale from the same amax;
+            // sb * f is positive and at most 448, so the code is in 1..126
             float sb = __fdiv_rn(a[u], 6.0f);
             if (sb <= min_value) sb = min_value;
-            const uint32_t code = e4m3x2_encode_hw(__fmul_rn(sb, f), 0.0f) & 0xFFu;
-            const float sq = __fdiv_rn(e4m3_decode(code), f);
-            const uint32_t c0 = e2m1x8_of_quotient(v[u], sq), c1 = e2m1x8_of_quotient(v[u] + 8, sq);
-            float o[16];
+            const uint32_t code = e4m3x2_encode_hw(__fmul_rn(sb, f), 0.0f) & 0x7Fu;
+            const float sq = sq_of[code];
+            const uint32_t pk = e2m1x8_of_quotient_r(v[u], sq, rsq_of[code]);
+            float e[8], o[8];
+            e2m1x8_decode_hw(pk, e);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                o[j] = __fmul_rn(e2m1_decode((c0 >> (4 * j)) & 15u), sq);
-                o[8 + j] = __fmul_rn(e2m1_decode((c1 >> (4 * j)) & 15u), sq);
-            }
-            store8(y + b * 16, o);
-            store8(y + b * 16 + 8, o + 8);
+            for (int j = 0; j < 8; ++j) o[j] = __fmaf_rn(e[j], sq, 0.0f);  // RN(e * sq); -0 -> +0
+            store8(y + c * 8, o);
         }
     }
 }
@@ -86,13 +99,13 @@ BSQ_API bsq_status bsq_fake_quantize_nvfp4_static(const void* x, bsq_dtype t, in
     const char* yb = (const char*)y;
     if (xb != yb && xb < yb + bytes && yb < xb + bytes)
         return fail(BSQ_ERR_INVALID_ARG, "%s: x and y overlap without being the same buffer", fn);
-    const int64_t nblocks = rows * K / 16;
+    const int64_t nchunks = rows * K / 8;
     cudaStream_t st = (cudaStream_t)stream;
     if (t == BSQ_BF16)
-        launch_fit<nv_static_fq_kernel<uint16_t, 2>>(nblocks, 2, st, (const uint16_t*)x, block_amax, global_amax,
-                                                      nblocks, (uint16_t*)y);
+        launch_fit<nv_static_fq_kernel<uint16_t, 4>>(nchunks, 4, st, (const uint16_t*)x, block_amax, global_amax,
+                                                      nchunks, (uint16_t*)y);
     else
-        launch_fit<nv_static_fq_kernel<float, 2>>(nblocks, 2, st, (const float*)x, block_amax, global_amax, nblocks,
+        launch_fit<nv_static_fq_kernel<float, 4>>(nchunks, 4, st, (const float*)x, block_amax, global_amax, nchunks,
                                                    (float*)y);
     return check_launch(fn);
 }
