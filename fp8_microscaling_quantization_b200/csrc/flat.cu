@@ -31,26 +31,25 @@ __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restric
     const int lane = threadIdx.x & 31;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t base = (int64_t)blockIdx.x * kThreads + (threadIdx.x & ~31); base < nchunks; base += U * stride) {
-        float v[U][8];
+        Raw8<T> raw[U];  // every chunk's load in flight before any arithmetic
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t c = base + u * stride + lane;
-            if (c < nchunks) load8(x + c * 8, v[u]);
-            else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
-            }
+            if (c < nchunks) raw[u].load(x + c * 8);
+            else raw[u].zero();
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t c = base + u * stride + lane;
-            const float amax_b = group_max<L>(amax8(v[u]));
+            float vu[8];
+            raw[u].get(vu);
+            const float amax_b = group_max<L>(amax8(vu));
             if (FMT == 1) {
                 const int e = mx_exponent(amax_b);
                 const float inv = exp2_int(-e);  // x * 2**-e == x / 2**e exactly
                 float q[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) q[j] = v[u][j] * inv;
+                for (int j = 0; j < 8; ++j) q[j] = vu[j] * inv;
                 const uint32_t packed = e2m1x8_encode_hw(q);
                 if (c < nchunks) {
                     reinterpret_cast<uint32_t*>(codes)[c] = packed;
@@ -61,10 +60,10 @@ __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restric
                 const int e = mx8_exponent(amax_b);
                 const float inv = exp2_int(-e);  // x * 2**-e == x / 2**e exactly
                 uint2 w;
-                w.x = e4m3x2_encode_hw(v[u][0] * inv, v[u][1] * inv) |
-                      (e4m3x2_encode_hw(v[u][2] * inv, v[u][3] * inv) << 16);
-                w.y = e4m3x2_encode_hw(v[u][4] * inv, v[u][5] * inv) |
-                      (e4m3x2_encode_hw(v[u][6] * inv, v[u][7] * inv) << 16);
+                w.x = e4m3x2_encode_hw(vu[0] * inv, vu[1] * inv) |
+                      (e4m3x2_encode_hw(vu[2] * inv, vu[3] * inv) << 16);
+                w.y = e4m3x2_encode_hw(vu[4] * inv, vu[5] * inv) |
+                      (e4m3x2_encode_hw(vu[6] * inv, vu[7] * inv) << 16);
                 if (c < nchunks) {
                     reinterpret_cast<uint2*>(codes)[c] = w;
                     if ((lane % L) == 0) scales[c / L] = (uint8_t)(e + 127);
@@ -73,10 +72,10 @@ __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restric
                 const float p = pow2_scale(amax_b, kE4M3Max);
                 const float inv = exp2_int(127 - f32_biased_exp(p));  // 1 / p, exact
                 uint2 w;
-                w.x = e4m3x2_encode_hw(v[u][0] * inv, v[u][1] * inv) |
-                      (e4m3x2_encode_hw(v[u][2] * inv, v[u][3] * inv) << 16);
-                w.y = e4m3x2_encode_hw(v[u][4] * inv, v[u][5] * inv) |
-                      (e4m3x2_encode_hw(v[u][6] * inv, v[u][7] * inv) << 16);
+                w.x = e4m3x2_encode_hw(vu[0] * inv, vu[1] * inv) |
+                      (e4m3x2_encode_hw(vu[2] * inv, vu[3] * inv) << 16);
+                w.y = e4m3x2_encode_hw(vu[4] * inv, vu[5] * inv) |
+                      (e4m3x2_encode_hw(vu[6] * inv, vu[7] * inv) << 16);
                 if (c < nchunks) {
                     reinterpret_cast<uint2*>(codes)[c] = w;
                     if ((lane % L) == 0) scales[c / L] = (uint8_t)f32_biased_exp(p);
