@@ -113,6 +113,23 @@ def traffic_from_profiles(*kernel_keys):
     return total
 
 
+# ------------------------------------------------------------ multi-rank --
+
+def job_time_ms(dist, region_ms, device):
+    """The job's time for the timed region: the maximum over ranks (each rank
+    times its own region with CUDA events; the slowest one ends the job)."""
+    import torch
+    t = torch.tensor([float(region_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world, step_bytes, ms_per_step):
+    """Whole-job throughput in GB/s: every rank runs its own copy of the
+    workload (weak scaling), so the job moves world * step_bytes per step."""
+    return world * step_bytes / (ms_per_step * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ clocks --
 
 class ClockSampler:
@@ -363,13 +380,11 @@ def main():
     clocks.stop()
     region_ms = ev_start.elapsed_time(ev_end)
     if world > 1:
-        t = torch.tensor([region_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        region_ms = float(t.item())
+        region_ms = job_time_ms(dist, region_ms, dev)
     ms_per_step = region_ms / steps
     qb, db, fb = mx_bytes()
     step_bytes = qb + db + fb
-    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    value = job_value(world, step_bytes, ms_per_step)
 
     kern = {}
     for key, nbytes in (("mx_quant", qb), ("mx_dequant_bf16", db), ("mx_dequant_fp32", fb)):
@@ -412,41 +427,62 @@ def main():
 
 def measure_e2e(torch, bsq, x_dev, stream, steps):
     """Quantize + dequantize through the C ABI with the step's input copied from
-    pinned host memory and every output copied back, inside the timed region."""
+    pinned host memory and every output copied back, inside the timed region.
+    Steps are pipelined over two buffer slots: step i's outputs stream back on
+    a copy stream while step i + 1's input streams in and its kernels run, so
+    the two PCIe directions overlap (the host-to-device copy, the kernels and
+    the device-to-host copy of every step are all inside the region)."""
     xh = x_dev.cpu().pin_memory()
-    xd = torch.empty_like(x_dev)
-    p = torch.empty((E, N, K // 2), dtype=torch.uint8, device=x_dev.device)
-    s = torch.empty((E, N, K // 32), dtype=torch.uint8, device=x_dev.device)
-    yb = torch.empty((E, N, K), dtype=torch.bfloat16, device=x_dev.device)
-    yf = torch.empty((E, N, K), dtype=torch.float32, device=x_dev.device)
-    ph, sh = torch.empty_like(p, device="cpu").pin_memory(), torch.empty_like(s, device="cpu").pin_memory()
-    ybh = torch.empty_like(yb, device="cpu").pin_memory()
-    yfh = torch.empty_like(yf, device="cpu").pin_memory()
+    dev = x_dev.device
+    xd = [torch.empty_like(x_dev) for _ in range(2)]
+    p = [torch.empty((E, N, K // 2), dtype=torch.uint8, device=dev) for _ in range(2)]
+    s = [torch.empty((E, N, K // 32), dtype=torch.uint8, device=dev) for _ in range(2)]
+    yb = [torch.empty((E, N, K), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    yf = [torch.empty((E, N, K), dtype=torch.float32, device=dev) for _ in range(2)]
+    ph = [torch.empty_like(p[0], device="cpu").pin_memory() for _ in range(2)]
+    sh = [torch.empty_like(s[0], device="cpu").pin_memory() for _ in range(2)]
+    ybh = [torch.empty_like(yb[0], device="cpu").pin_memory() for _ in range(2)]
+    yfh = [torch.empty_like(yf[0], device="cpu").pin_memory() for _ in range(2)]
+    out_stream = torch.cuda.Stream(device=dev)
+    computed = [torch.cuda.Event() for _ in range(2)]
+    drained = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        xd.copy_(xh, non_blocking=True)
-        bsq.bsq_quantize_mxfp4(xd, packed=p, scales=s)
-        bsq.bsq_dequantize_mxfp4(p, s, y=yb)
-        bsq.bsq_dequantize_mxfp4(p, s, y=yf, out_dtype=bsq.DType.FP32)
-        ph.copy_(p, non_blocking=True)
-        sh.copy_(s, non_blocking=True)
-        ybh.copy_(yb, non_blocking=True)
-        yfh.copy_(yf, non_blocking=True)
+    def step(i):
+        k = i % 2
+        if i >= 2:
+            stream.wait_event(drained[k])  # slot k's previous outputs are on the host
+        with torch.cuda.stream(stream):
+            xd[k].copy_(xh, non_blocking=True)
+            bsq.bsq_quantize_mxfp4(xd[k], packed=p[k], scales=s[k])
+            bsq.bsq_dequantize_mxfp4(p[k], s[k], y=yb[k])
+            bsq.bsq_dequantize_mxfp4(p[k], s[k], y=yf[k], out_dtype=bsq.DType.FP32)
+        computed[k].record(stream)
+        out_stream.wait_event(computed[k])
+        with torch.cuda.stream(out_stream):
+            ph[k].copy_(p[k], non_blocking=True)
+            sh[k].copy_(s[k], non_blocking=True)
+            ybh[k].copy_(yb[k], non_blocking=True)
+            yfh[k].copy_(yf[k], non_blocking=True)
+        drained[k].record(out_stream)
 
-    one()
+    for i in range(2):
+        step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
+    out_stream.wait_event(e0)
+    for i in range(steps):
+        step(i)
+    out_stream.wait_stream(stream)
+    e1.record(out_stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
     qb, db, fb = mx_bytes()
     h2d = xh.numel() * 2
-    d2h = ph.numel() + sh.numel() + ybh.numel() * 2 + yfh.numel() * 4
+    d2h = ph[0].numel() + sh[0].numel() + ybh[0].numel() * 2 + yfh[0].numel() * 4
     return {"value": round((qb + db + fb) / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3)}
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
+            "note": "pinned host buffers; two slots, input copy + kernels on one stream, output copy on another"}
 
 
 # ------------------------------------------------------------- sub-measures -
@@ -513,17 +549,22 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
         g.manual_seed(20260007)
         nbk, bt, hd = 1024, 64, 8
         rows = bt * hd
-        vals = [torch.randint(0, 256, (rows, 64), generator=g, device=dev, dtype=torch.uint8) for _ in range(nbk)]
-        scs = [torch.randint(0, 0x7E, (rows, 8), generator=g, device=dev, dtype=torch.uint8) for _ in range(nbk)]
-        ams = [torch.rand((1,), generator=g, device=dev) * 100 for _ in range(nbk)]
+        # separate, non-contiguous blocks: views into three allocations with a
+        # gap after every block (three launches to fill instead of thousands)
+        vpool = torch.randint(0, 256, (nbk, rows + 16, 64), generator=g, device=dev, dtype=torch.uint8)
+        spool = torch.randint(0, 0x7E, (nbk, rows + 16, 8), generator=g, device=dev, dtype=torch.uint8)
+        apool = torch.rand((nbk, 4), generator=g, device=dev) * 100
+        vals = [vpool[i, :rows] for i in range(nbk)]
+        scs = [spool[i, :rows] for i in range(nbk)]
+        ams = [apool[i, :1] for i in range(nbk)]
         table = bsq.kv_block_table(vals, scs, ams)
         yk = torch.empty((1, nbk * bt, hd, 128), dtype=torch.bfloat16, device=dev)
         n = nbk * rows * 128
         out["kv_cache_nvfp4_1024x64x8x128"] = {
             "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_kv_cache_nvfp4(table, nbk, bt, hd, y=yk), 10, True),
                                    n // 2 + n // 16 + 4 * nbk + 2 * n, "kv_dequant_bf16"),
-            "note": "1024 separately allocated blocks of 64 tokens x 8 heads x 128; L2 flushed before every launch"}
-        del vals, scs, ams, table, yk
+            "note": "1024 non-contiguous blocks of 64 tokens x 8 heads x 128; L2 flushed before every launch"}
+        del vals, scs, ams, vpool, spool, apool, table, yk
 
     if want("cache"):
         g = torch.Generator(device=dev)
