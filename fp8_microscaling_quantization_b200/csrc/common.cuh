@@ -133,9 +133,6 @@ __device__ __forceinline__ void build_e2m1_lut(float2* lut) {
 
 // ----------------------------------------------------------------- NVFP4 ----
 
-// Quantize one 8-element chunk whose block partner is lane ^ 1, given the
-// row scale g (g == 0: zero row).  Returns the packed 4 bytes; *scale_byte
-// receives the block's e4m3 scale.
 // e2m1 codes of RN(v[j] / d) for 8 values, bit-exact, mostly without a
 // division.  With r = RN(1/d), q = RN(v * r) lies within 1.5 * 2**-23 * |q| of
 // RN(v / d) (two roundings of 2**-24 each, d and r normal).  The e2m1 rounding
@@ -169,20 +166,6 @@ __device__ __forceinline__ uint32_t e2m1x8_of_quotient_r(const float v[8], float
     return e2m1x8_encode_hw(q);
 }
 
-// Quantize one 8-element chunk whose block partner is lane ^ 1, given the
-// row scale g (g == 0: zero row).  Returns the packed 4 bytes; *scale_byte
-// receives the block's e4m3 scale.
-__device__ __forceinline__ uint32_t nv_quant_chunk(const float v[8], float g, uint32_t* scale_byte) {
-    const float amax_b = group_max<2>(amax8(v));
-    if (g == 0.0f) {
-        *scale_byte = 0u;
-        return 0u;
-    }
-    const uint32_t s = nv_scale_byte(amax_b, g);
-    const float d = __fmul_rn(e4m3_decode(s), g);
-    *scale_byte = s;
-    return e2m1x8_of_quotient(v, d);
-}
 
 // ---- one lane per 16-element NVFP4 block --------------------------------
 
