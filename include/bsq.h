@@ -3,10 +3,13 @@
  * NVIDIA B200 (sm_100a).
  *
  * Formats (NeMo AutoModel API pages "nemo_automodel.components.quantization.nvfp4",
- * "...quantization.mxfp4" and "...models.deepseek_v41.quantization"):
+ * "...quantization.mxfp4" and "...models.deepseek_v41.quantization"; the
+ * ModelOpt tensor_quantizer page for MXFP8 and the static two-level NVFP4
+ * quantizer; the NeMo AutoModel model-filter page for the NVFP4 KV cache):
  *   NVFP4 -- e2m1 codes, one float8_e4m3fn scale per 16 columns and one fp32
  *            scale per row (or per tensor, the ModelOpt checkpoint layout).
  *   MXFP4 -- e2m1 codes, one float8_e8m0fnu scale per 32 columns.
+ *   MXFP8 -- float8_e4m3fn codes, one float8_e8m0fnu scale per 32 columns.
  *   FP8   -- float8_e4m3fn codes with a power-of-two block scale, stored as an
  *            e8m0 exponent byte per block.
  * Two e2m1 codes share a byte: the even column in the low nibble, the odd
@@ -16,9 +19,13 @@
  *   - Tensors are contiguous and row-major; "rows" is the product of all
  *     leading dimensions and K (or C) the last dimension.
  *   - Every data pointer is a DEVICE pointer, owned by the caller.  The
- *     library never allocates or frees device memory and keeps no state
- *     between calls; outputs are written in place, so buffer addresses stay
- *     stable (CUDA graph friendly).  Inputs are never modified.
+ *     library never allocates or frees device memory and keeps no device
+ *     data between calls (the one exception, the file-scope scratch of
+ *     bsq_quantize_nvfp4_tensor_noalloc, is described there); it caches only
+ *     host-side facts (SM count, occupancy, the tensor-map encoder).  Outputs
+ *     are written in place, so buffer addresses stay stable (CUDA graph
+ *     friendly).  Inputs are never modified, except that
+ *     bsq_fake_quantize_nvfp4_static may be asked to write over its input.
  *   - Work is enqueued on `stream` and is asynchronous.  Only argument
  *     validation runs on the host; a rejected call launches nothing.
  *   - Return value: BSQ_OK, or an error code; bsq_last_error() returns a
