@@ -96,9 +96,9 @@ __device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg,
 #pragma unroll
         for (int j = 0; j < 8; ++j) q[j] = v[j] * inv;
         e2m1x8_decode_hw(e2m1x8_encode_hw(q), e);
-        // e * p is exact; adding +0 turns code 8's -0 into the table's +0
+        // e * p is exact
 #pragma unroll
-        for (int j = 0; j < 8; ++j) out[j] = __fmaf_rn(e[j], p, 0.0f);
+        for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(e[j], p);
     } else {
         if (g == 0.0f) {
 #pragma unroll
@@ -110,7 +110,7 @@ __device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg,
             e2m1x8_decode_hw(e2m1x8_of_quotient(v, d), e);
             // (e2m1 * s) is exact (and +0 for code 8), then one rounding by g
 #pragma unroll
-            for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(__fmaf_rn(e[j], s, 0.0f), g);
+            for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(__fmul_rn(e[j], s), g);
         }
     }
 }

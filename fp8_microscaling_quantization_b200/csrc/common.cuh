@@ -125,12 +125,6 @@ __device__ __forceinline__ uint32_t nv_scale_byte(float amax_b, float g) {
     return e4m3_encode_sw(t);
 }
 
-// e2m1 byte -> (value of low nibble, value of high nibble), built per CTA.
-__device__ __forceinline__ void build_e2m1_lut(float2* lut) {
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) lut[b] = make_float2(e2m1_decode(b & 15), e2m1_decode(b >> 4));
-    __syncthreads();
-}
-
 // ----------------------------------------------------------------- NVFP4 ----
 
 // e2m1 codes of RN(v[j] / d) for 8 values, bit-exact, mostly without a

@@ -88,9 +88,8 @@ __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restric
 // Dequantize (all formats).  Item = the EPI consecutive output elements of
 // one lane: 8 for bf16 output (one 16-byte store) and 4 for fp32 output (one
 // 16-byte store), so consecutive lanes write consecutive 16-byte pieces and a
-// warp store instruction covers one contiguous 512-byte span.  FP4 codes are
-// decoded through a 256-entry byte -> (low value, high value) table in shared
-// memory; e4m3 codes through the hardware cvt (exact).
+// warp store instruction covers one contiguous 512-byte span.  e2m1 and e4m3
+// codes are decoded by the hardware conversions (exact).
 //   FMT_MX : y = e2m1 * 2**(scale - 127)
 //   FMT_NV : y = (e2m1 * e4m3(scale)) * g[row], row = block / bpr
 //   FMT_FP8: y = e4m3 * 2**(scale - 127)
@@ -103,8 +102,6 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __rest
                                                            int64_t nitems, TOUT* __restrict__ y) {
     constexpr int EPI = (sizeof(TOUT) == 2) ? 8 : 4;         // elements per item
     constexpr int CB = (FMT == FMT_FP8) ? EPI : EPI / 2;     // code bytes per item
-    __shared__ float2 lut[256];
-    if (FMT != FMT_FP8) build_e2m1_lut(lut);
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t base = (int64_t)blockIdx.x * kThreads + threadIdx.x; base < nitems; base += U * stride) {
         uint32_t w0[U], w1[U], sc[U];
@@ -143,17 +140,13 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __rest
                 }
             } else {
                 const float s = (FMT == FMT_MX) ? e8m0_decode(sc[u]) : e4m3_decode(sc[u]);
+                // e2m1 * s is exact (a power of two for MXFP4, 6 significant
+                // bits for NVFP4); the decode already gives code 8 as +0
+                float e[8];
+                e2m1x8_decode_hw(w0[u], e);  // fp32 output: the first EPI = 4 are used
 #pragma unroll
-                for (int i = 0; i < EPI / 2; ++i) {
-                    const float2 t = lut[(w0[u] >> (8 * i)) & 0xFFu];
-                    if (FMT == FMT_MX) {
-                        v[2 * i] = t.x * s;
-                        v[2 * i + 1] = t.y * s;
-                    } else {
-                        v[2 * i] = __fmul_rn(__fmul_rn(t.x, s), gr[u]);
-                        v[2 * i + 1] = __fmul_rn(__fmul_rn(t.y, s), gr[u]);
-                    }
-                }
+                for (int j = 0; j < EPI; ++j)
+                    v[j] = (FMT == FMT_MX) ? __fmul_rn(e[j], s) : __fmul_rn(__fmul_rn(e[j], s), gr[u]);
             }
             TOUT* dst = y + it * EPI;
             if (sizeof(TOUT) == 2) {

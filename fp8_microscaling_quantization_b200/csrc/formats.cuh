@@ -118,8 +118,8 @@ __device__ __forceinline__ uint32_t e2m1x8_encode_hw(const float v[8]) {
 
 // Four bytes of packed e2m1 codes -> eight binary32 values (code 2i + j from
 // nibble j of byte i), by the hardware conversion to f16x2 and f16 -> f32
-// (both exact).  Code 8 gives -0.0 here; a caller that needs the table's
-// +0.0 adds +0.0 (fma(v, s, 0.0f) rounds v * s once and turns -0 into +0).
+// (both exact).  The conversion gives -0.0 for code 8; adding +0.0 turns that
+// into the table's +0.0 and leaves every other value unchanged.
 __device__ __forceinline__ void e2m1x8_decode_hw(uint32_t w, float v[8]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -130,20 +130,11 @@ __device__ __forceinline__ void e2m1x8_decode_hw(uint32_t w, float v[8]) {
             : "=r"(h2)
             : "r"(w >> (8 * i)));
         const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
-        v[2 * i] = f.x;
-        v[2 * i + 1] = f.y;
+        v[2 * i] = __fadd_rn(f.x, 0.0f);
+        v[2 * i + 1] = __fadd_rn(f.y, 0.0f);
     }
 }
 
-// e2m1 code -> binary32.  Magnitude m: 0 and 1 are 0 and 0.5; m >= 2 is
-// (1 + (m & 1) / 2) * 2**((m >> 1) - 1).  Code 8 decodes to +0.0.
-__device__ __forceinline__ float e2m1_decode(uint32_t c) {
-    uint32_t m = c & 7u;
-    uint32_t bits = (m >= 2u) ? ((((m >> 1) + 126u) << 23) | ((m & 1u) << 22))
-                              : (m == 1u ? 0x3F000000u : 0u);
-    if ((c & 8u) && m) bits |= 0x80000000u;
-    return __uint_as_float(bits);
-}
 
 // e8m0 byte -> 2**(code - 127) as binary32 (code 0 is the subnormal 2**-127,
 // 0xFF is NaN).

@@ -88,9 +88,9 @@ __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const uint8_t* con
             const float s = e4m3_decode(sc[u]);
             float e[8], v[8];
             e2m1x8_decode_hw(w[u], e);  // fp32 output: only the first 4 are used
-            // (e2m1 * s) is exact, and +0 for code 8; then one rounding by g
+            // e2m1 * s first (exact), then one rounding by g
 #pragma unroll
-            for (int i = 0; i < EPI; ++i) v[i] = __fmul_rn(__fmaf_rn(e[i], s, 0.0f), gr[u]);
+            for (int i = 0; i < EPI; ++i) v[i] = __fmul_rn(__fmul_rn(e[i], s), gr[u]);
             TOUT* dst = y + it * EPI;
             if (sizeof(TOUT) == 2) {
                 uint4 o4;

@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kThreads) nv_static_fq_kernel(const T* __restr
             float e[8], o[8];
             e2m1x8_decode_hw(pk, e);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) o[j] = __fmaf_rn(e[j], sq, 0.0f);  // RN(e * sq); -0 -> +0
+            for (int j = 0; j < 8; ++j) o[j] = __fmul_rn(e[j], sq);
             store8(y + c * 8, o);
         }
     }

@@ -85,3 +85,25 @@ def test_kv_cache_empty_and_rejects(B):
     with pytest.raises(B.BsqError):
         B.bsq_dequantize_kv_cache_nvfp4((t, t, t), -1, 64, 8, y=y)
     torch.cuda.synchronize()
+
+
+def test_kv_cache_dequant_all_scale_codes(B, oracle):
+    """Arbitrary bytes in the cache: every e2m1 code next to every finite e4m3
+    scale code, negative scales included (the sign of a zero product follows
+    the scale), so the decode order and signed zeros are checked bit for bit."""
+    rng = np.random.default_rng(21)
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    block_tokens, heads = 16, 2
+    rows = block_tokens * heads
+    vals, scs, amax = [], [], []
+    for b in range(8):
+        vals.append(rng.integers(0, 256, (rows, 64), dtype=np.uint8))
+        scs.append(codes[rng.integers(0, codes.size, (rows, 8))])
+        amax.append(np.float32(rng.uniform(1e-3, 1e4)))
+    scs[0] = np.resize(codes, (rows, 8))  # block 0 holds every scale code
+    amax = np.array(amax, np.float32)
+    _, table = to_device(B, vals, scs, amax)
+    for dt, odt in ((B.DType.BF16, oracle.BF16), (B.DType.FP32, oracle.F32)):
+        y = B.bsq_dequantize_kv_cache_nvfp4(table, len(vals), block_tokens, heads, out_dtype=dt)
+        assert_bits_equal(host_bits(y), oracle.dequantize_kv_cache_nvfp4(vals, scs, amax, block_tokens, heads,
+                                                                          out_dtype=odt), f"kv all codes {dt}")
