@@ -9,16 +9,20 @@
 // to the output dtype.  Block b fills output tokens [b * block_tokens,
 // (b + 1) * block_tokens), so the output of block b is one contiguous range.
 //
-// One fused launch for every block: an item is 8 outputs (bf16, one 16-byte
-// store) or 4 (fp32), consecutive lanes take consecutive items, and each warp
-// walks a run of 32 * U items.  The block of an item comes from a
-// constant-divisor multiply; a lane loads the block's pointers and global
-// scale only when its item enters another block, so the load pipe carries
-// little beyond the codes, the scale bytes and the stores.  e2m1 codes are
-// decoded by the hardware e2m1 -> f16x2 conversion.
+// One fused launch for every block.  The work is cut into units of
+// kThreads * kKvUnroll consecutive items (an item is 8 outputs, one 16-byte
+// bf16 store, or 4 fp32 outputs) that never straddle two cache blocks; a CTA
+// takes units in turn and each thread handles kKvUnroll items kThreads apart,
+// so a warp's loads and stores are contiguous.  A unit's block pointers and
+// amax are the same address for every thread of the CTA, and they are loaded
+// while the previous unit runs, so the codes of a unit are requested without
+// first waiting for a pointer.  e2m1 codes are decoded by the hardware
+// e2m1 -> f16x2 conversion.
 #include "common.cuh"
 
 namespace bsq {
+
+constexpr int kKvUnroll = 8;  // items per thread per unit
 
 // The block pointers sit in device memory where the host cannot check them:
 // word loads go through these, which fall back to byte loads when a pointer
@@ -43,55 +47,58 @@ template <typename TOUT, int U>
 __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const uint8_t* const* __restrict__ values,
                                                               const uint8_t* const* __restrict__ scales,
                                                               const float* const* __restrict__ amax,
-                                                              FastDiv items_per_block, int64_t nitems,
-                                                              TOUT* __restrict__ y) {
+                                                              FastDiv units_per_block, uint32_t items_per_block,
+                                                              int64_t nunits, TOUT* __restrict__ y) {
     constexpr int EPI = (sizeof(TOUT) == 2) ? 8 : 4;  // outputs per item
-    constexpr int RUN = 32 * U;                       // items of one warp's run
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
-    // the block's pointers and global scale, reloaded only when a lane's item
-    // moves into another block (a run lies in one block unless it straddles
-    // a boundary)
-    uint32_t cur = 0xFFFFFFFFu;
-    const uint8_t* vb = nullptr;
-    const uint8_t* sb = nullptr;
-    float g = 0.0f;
-    for (int64_t run = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); run * RUN < nitems;
-         run += warps) {
-        uint32_t w[U], sc[U];
-        float gr[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t it = run * RUN + u * 32 + lane;  // consecutive lanes, consecutive items
-            w[u] = sc[u] = 0u;
-            gr[u] = 0.0f;
-            if (it < nitems) {
-                const uint32_t b = fdiv((uint32_t)it, items_per_block);
-                if (b != cur) {
-                    cur = b;
-                    vb = values[b];
-                    sb = scales[b];
-                    g = __fdiv_rn(ld_f32_any(amax[b]), 2688.0f);
-                }
-                const uint32_t o = (uint32_t)it - b * items_per_block.d;  // item within the block
-                w[u] = ld_codes(vb, o, EPI / 2);
-                // element o * EPI of the block: row (o * EPI) / 128, scale column ((o * EPI) % 128) / 16,
-                // i.e. scale byte (o * EPI) / 16 of the row-major [rows, 8] scales
-                sc[u] = sb[(o * EPI) >> 4];
-                gr[u] = g;
+    constexpr int UNIT = kThreads * U;                // items per unit
+    int64_t unit = blockIdx.x;
+    if (unit >= nunits) return;
+    uint32_t b = fdiv((uint32_t)unit, units_per_block);
+    const uint8_t* vb = values[b];
+    const uint8_t* sb = scales[b];
+    float a = ld_f32_any(amax[b]);
+    for (; unit < nunits; unit += gridDim.x) {
+        const uint32_t c = (uint32_t)unit - b * units_per_block.d;
+        const float g = __fdiv_rn(a, 2688.0f);
+        // the next unit's block pointers and amax, loaded while this unit runs
+        const int64_t nxt = unit + gridDim.x;
+        uint32_t nb = b;
+        const uint8_t* nvb = vb;
+        const uint8_t* nsb = sb;
+        float na = a;
+        if (nxt < nunits) {
+            nb = fdiv((uint32_t)nxt, units_per_block);
+            if (nb != b) {
+                nvb = values[nb];
+                nsb = scales[nb];
+                na = ld_f32_any(amax[nb]);
             }
         }
+        const uint32_t o0 = c * UNIT + threadIdx.x;  // item within the block
+        uint32_t w[U], sc[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t it = run * RUN + u * 32 + lane;
-            if (it >= nitems) continue;
+            const uint32_t o = o0 + u * kThreads;
+            w[u] = sc[u] = 0u;
+            if (o < items_per_block) {
+                w[u] = ld_codes(vb, o, EPI / 2);
+                // element o * EPI of the block: scale byte (o * EPI) / 16 of
+                // the row-major [rows, 8] scales
+                sc[u] = sb[(o * EPI) >> 4];
+            }
+        }
+        TOUT* yb = y + (int64_t)b * items_per_block * EPI;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t o = o0 + u * kThreads;
+            if (o >= items_per_block) continue;
             const float s = e4m3_decode(sc[u]);
             float e[8], v[8];
             e2m1x8_decode_hw(w[u], e);  // fp32 output: only the first 4 are used
             // e2m1 * s first (exact), then one rounding by g
 #pragma unroll
-            for (int i = 0; i < EPI; ++i) v[i] = __fmul_rn(__fmul_rn(e[i], s), gr[u]);
-            TOUT* dst = y + it * EPI;
+            for (int i = 0; i < EPI; ++i) v[i] = __fmul_rn(__fmul_rn(e[i], s), g);
+            TOUT* dst = yb + (int64_t)o * EPI;
             if (sizeof(TOUT) == 2) {
                 uint4 o4;
                 o4.x = pack_bf16x2(v[0], v[1]);
@@ -103,6 +110,10 @@ __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const uint8_t* con
                 __stcs(reinterpret_cast<float4*>(dst), make_float4(v[0], v[1], v[2], v[3]));
             }
         }
+        b = nb;
+        vb = nvb;
+        sb = nsb;
+        a = na;
     }
 }
 
@@ -123,13 +134,19 @@ BSQ_API bsq_status bsq_dequantize_kv_cache_nvfp4(const uint8_t* const* values, c
     const int epi = (yt == BSQ_BF16) ? 8 : 4;
     const int64_t items_per_block = block_tokens * heads * 128 / epi;
     const int64_t nitems = nblocks * items_per_block;
-    if (items_per_block > 0x7FFFFFFF || nitems > 0xFFFFFFFFll)
-        return fail(BSQ_ERR_UNSUPPORTED, "%s: more than 2**32 output items", fn);
-    const FastDiv ipb = make_fastdiv((uint32_t)items_per_block);
+    if (items_per_block * epi > 0xFFFFFFFFll || nitems > 0xFFFFFFFFll)
+        return fail(BSQ_ERR_UNSUPPORTED, "%s: more than 2**32 outputs per block or items in all", fn);
+    constexpr int kUnit = kThreads * kKvUnroll;
+    const int64_t upb = (items_per_block + kUnit - 1) / kUnit;  // units per cache block
+    const int64_t nunits = nblocks * upb;
+    const FastDiv fupb = make_fastdiv((uint32_t)upb);
+    const uint32_t ipb = (uint32_t)items_per_block;
     cudaStream_t st = (cudaStream_t)stream;
     if (yt == BSQ_BF16)
-        launch_fit<kv_dequant_kernel<uint16_t, 8>>(nitems, 8, st, values, scales, amax, ipb, nitems, (uint16_t*)y);
+        launch_fit_ctas<kv_dequant_kernel<uint16_t, kKvUnroll>>(nunits, st, values, scales, amax, fupb, ipb, nunits,
+                                                                (uint16_t*)y);
     else
-        launch_fit<kv_dequant_kernel<float, 8>>(nitems, 8, st, values, scales, amax, ipb, nitems, (float*)y);
+        launch_fit_ctas<kv_dequant_kernel<float, kKvUnroll>>(nunits, st, values, scales, amax, fupb, ipb, nunits,
+                                                             (float*)y);
     return check_launch(fn);
 }
