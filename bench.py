@@ -578,6 +578,11 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
             y = torch.empty_like(x)
             nb = 2 * 2 * x.numel()
             res[name] = rec(timed(lambda: bsq.bsq_quantize_cache(x, fmt, blk, y=y), 30, True), nb, "cache_" + name)
+            # the latency floor at this size: a device-to-device copy of the
+            # same bytes, timed the same way
+            copy_ms = timed(lambda: y.copy_(x), 30, True)
+            res[name]["same_size_copy_us"] = round(copy_ms * 1e3, 2)
+            res[name]["frac_of_copy"] = round(copy_ms * 1e3 / res[name]["us"], 4)
         gsrc = torch.randn((4, 8192, 512), generator=g, device=dev).to(torch.bfloat16)
         gdst = torch.empty_like(gsrc)
         res["ste_backward_aliased"] = {"us": 0.0, "bytes": 0, "note": "identity: no launch"}

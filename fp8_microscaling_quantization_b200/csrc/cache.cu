@@ -117,9 +117,12 @@ __device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg,
 
 // FP8 / MXFP4 fake-quant when every row is a whole number of blocks and
 // 16-byte aligned: the blocks tile the flat tensor, so this is a flat stream
-// with U chunks in flight per lane.
+// with U chunks in flight per lane.  Bounded to 32 registers so that 8 CTAs
+// fit on an SM: the tensors of this path are 8-70 MB, and at that size more
+// resident warps (more loads in flight at the start) beat more chunks per
+// lane.
 template <typename T, int FMT, int BLOCK, int U>
-__global__ void __launch_bounds__(kThreads) cache_flat_kernel(const T* __restrict__ x, T* __restrict__ y,
+__global__ void __launch_bounds__(kThreads, 8) cache_flat_kernel(const T* __restrict__ x, T* __restrict__ y,
                                                               int64_t nchunks) {
     constexpr int L = BLOCK / 8;
     const int lane = threadIdx.x & 31;
@@ -217,7 +220,7 @@ static void launch_cache_s(const T* x, T* y, int64_t rows, int64_t C, cudaStream
     const int64_t cpr = ((C + BLOCK - 1) / BLOCK) * (BLOCK / 8);
     if (FMT != BSQ_NVFP4 && VEC && C % BLOCK == 0) {
         const int64_t nchunks = rows * C / 8;
-        launch_fit<cache_flat_kernel<T, FMT, BLOCK, 4>>(nchunks, 4, st, x, y, nchunks);
+        launch_fit<cache_flat_kernel<T, FMT, BLOCK, 2>>(nchunks, 2, st, x, y, nchunks);
         return;
     }
     int S = 2;
