@@ -107,3 +107,16 @@ def test_kv_cache_dequant_all_scale_codes(B, oracle):
         y = B.bsq_dequantize_kv_cache_nvfp4(table, len(vals), block_tokens, heads, out_dtype=dt)
         assert_bits_equal(host_bits(y), oracle.dequantize_kv_cache_nvfp4(vals, scs, amax, block_tokens, heads,
                                                                           out_dtype=odt), f"kv all codes {dt}")
+
+
+def test_kv_cache_long_blocks(B, oracle):
+    """Two blocks of 16384 tokens x 8 heads: each block is 1024 work units of
+    the kernel, more than the CTAs resident on the device, so a CTA's next
+    unit often lies in the block it is working on (the pointers it
+    prefetched are the current ones) and sometimes in the other block."""
+    vals, scs, amax = make_cache(oracle, 2, 16384, 8, seed=31)
+    _, table = to_device(B, vals, scs, amax)
+    for dt, odt in ((B.DType.BF16, oracle.BF16), (B.DType.FP32, oracle.F32)):
+        y = B.bsq_dequantize_kv_cache_nvfp4(table, 2, 16384, 8, out_dtype=dt)
+        want = oracle.dequantize_kv_cache_nvfp4(vals, scs, amax, 16384, 8, out_dtype=odt)
+        assert_bits_equal(host_bits(y), want, f"kv long blocks {dt}")
