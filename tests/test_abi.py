@@ -113,3 +113,52 @@ def test_tensor_scratch_size(lib):
     rc = lib.bsq_quantize_nvfp4_tensor(FAKE, 0, I64(7168), I64(18432), FAKE, FAKE, FAKE, FAKE,
                                        ctypes.c_size_t(0), None)
     assert rc == INVALID and "scratch" in _err(lib)
+
+
+def test_kv_cache_host_checks(lib):
+    P = ctypes.c_void_p
+    # no blocks (or an empty block shape): nothing to do, even with null pointers
+    assert lib.bsq_dequantize_kv_cache_nvfp4(None, None, None, I64(0), I64(64), I64(8), None, 0, None) == 0
+    assert lib.bsq_dequantize_kv_cache_nvfp4(None, None, None, I64(4), I64(0), I64(8), None, 0, None) == 0
+    assert lib.bsq_dequantize_kv_cache_nvfp4(FAKE, FAKE, FAKE, I64(-1), I64(64), I64(8), FAKE, 0, None) == INVALID
+    assert lib.bsq_dequantize_kv_cache_nvfp4(FAKE, None, FAKE, I64(4), I64(64), I64(8), FAKE, 0, None) == INVALID
+    # the pointer arrays hold 8-byte pointers; the output takes 16-byte stores
+    assert lib.bsq_dequantize_kv_cache_nvfp4(P(0x10004), FAKE, FAKE, I64(4), I64(64), I64(8), FAKE, 0,
+                                             None) == INVALID
+    rc = lib.bsq_dequantize_kv_cache_nvfp4(FAKE, FAKE, FAKE, I64(4), I64(64), I64(8), P(0x10008), 0, None)
+    assert rc == INVALID and "misaligned" in _err(lib)
+    # 2**33 outputs in one block: beyond the kernel's 32-bit in-block index
+    rc = lib.bsq_dequantize_kv_cache_nvfp4(FAKE, FAKE, FAKE, I64(1), I64(1 << 25), I64(2), FAKE, 0, None)
+    assert rc == UNSUPPORTED and "2**32" in _err(lib)
+    assert lib.bsq_dequantize_kv_cache_nvfp4(FAKE, FAKE, FAKE, I64(4), I64(64), I64(8), FAKE, 5, None) == UNSUPPORTED
+
+
+def test_static_fake_quant_host_checks(lib):
+    P = ctypes.c_void_p
+    f = lib.bsq_fake_quantize_nvfp4_static
+    assert f(FAKE, 0, I64(4), I64(24), FAKE, FAKE, P(0x90000), None) == INVALID  # K not a multiple of 16
+    assert f(None, 0, I64(0), I64(32), None, None, None, None) == 0  # empty
+    assert f(FAKE, 0, I64(4), I64(32), None, FAKE, P(0x90000), None) == INVALID  # no block amax
+    assert f(FAKE, 0, I64(4), I64(32), FAKE, FAKE, P(0x90008), None) == INVALID  # misaligned output
+    rc = f(FAKE, 0, I64(4), I64(32), FAKE, FAKE, P(0x10000 + 32), None)  # partial overlap (in place is fine)
+    assert rc == INVALID and "overlap" in _err(lib)
+
+
+def test_mxfp8_host_checks(lib):
+    assert lib.bsq_quantize_mxfp8(FAKE, 0, I64(4), I64(48), FAKE, FAKE, None) == INVALID  # K % 32
+    assert lib.bsq_dequantize_mxfp8(FAKE, FAKE, I64(4), I64(48), FAKE, 0, None) == INVALID
+    assert lib.bsq_quantize_mxfp8(None, 0, I64(0), I64(64), None, None, None) == 0
+
+
+def test_grouped_mm_host_checks(lib):
+    g = lib.bsq_grouped_mm_fp4
+    MX, NV, FWD, BWD = 1, 2, 0, 1
+    args = lambda fmt, d, E, T, N, K, err=FAKE, rs=FAKE: (fmt, d, FAKE, FAKE, FAKE, rs, FAKE, E, I64(T), I64(N),
+                                                          I64(K), FAKE, err, None)
+    assert g(*args(0, FWD, 4, 256, 256, 256)) == UNSUPPORTED  # FP8 weights are not a GEMM format here
+    assert g(*args(MX, 7, 4, 256, 256, 256)) == INVALID  # direction
+    assert g(*args(MX, FWD, 0, 256, 256, 256)) == INVALID  # no experts
+    assert g(*args(MX, FWD, 4, 256, 256, 200)) == UNSUPPORTED  # K not a multiple of 64
+    assert g(*args(MX, FWD, 4, 256, 256, 256, err=None)) == INVALID  # the error word is required
+    assert g(*args(NV, FWD, 4, 256, 256, 256, rs=None)) == INVALID  # NVFP4 needs its row scales
+    assert g(*args(MX, FWD, 4, 0, 256, 256)) == 0  # no tokens: nothing to do
