@@ -1,0 +1,178 @@
+"""The division-free roundings behind the kernels' bit-exact NVFP4 codes,
+replayed on the CPU in binary32 and compared with the plain divisions.
+
+Element code.  The code is the e2m1 rounding of RN(x / d).  Instead of
+dividing, one can form q = RN(x * RN(1/d)), which lies within 1.5 * 2**-23
+* |q| of RN(x / d), and round the two brackets RN(q * (1 -+ 2**-21)).  e2m1
+rounding is monotone, so when both brackets give the same code, that code is
+RN(x / d)'s.  When they differ, or d is outside [2**-125, 2**125], the
+division is done.
+
+Block scale code.  The code is e4m3(max(RN(RN(a / 6) / g), 2**-9)).  The
+same argument applies to t1 = RN(RN(a * RN(1/6)) * RN(1/g)), with brackets
+(1 -+ 2**-20) clamped at 2**-9, when g and 1/g are normal and a is 0 or at
+least 2**-120.
+
+Here both shortcuts run in numpy binary32, which rounds each operation to
+nearest even and keeps subnormals. Their codes come from the oracle's
+roundings and are compared with the oracle's rounding of the plain
+quotients, on random operands and on operands placed within a few ulps of
+every rounding boundary.  CPU only.
+"""
+import numpy as np
+import pytest
+
+F = np.float32
+LO21, HI21 = F(1 - 2.0 ** -21), F(1 + 2.0 ** -21)
+LO20, HI20 = F(1 - 2.0 ** -20), F(1 + 2.0 ** -20)
+MIN_SCALE = F(2.0 ** -9)
+E2M1_MIDPOINTS = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+
+
+def element_codes_by_bracket(oracle, x, d):
+    """(code, decided): the bracket code and whether the brackets agreed."""
+    with np.errstate(over="ignore", under="ignore", invalid="ignore"):
+        r = F(1) / d
+        q = x * r
+        lo, hi = q * LO21, q * HI21
+    clo, chi = oracle.e2m1_round(lo), oracle.e2m1_round(hi)
+    in_range = (d >= F(2.0 ** -125)) & (d <= F(2.0 ** 125))
+    return clo, (clo == chi) & in_range
+
+
+def element_codes_by_division(oracle, x, d):
+    with np.errstate(over="ignore", under="ignore", divide="ignore", invalid="ignore"):
+        return oracle.e2m1_round(x / d)
+
+
+def e4m3_values(oracle):
+    codes = np.array([c for c in range(1, 127)], dtype=np.uint8)  # positive finite
+    return np.array([oracle.e4m3_val(int(c)) for c in codes], dtype=np.float32)
+
+
+def check_elements(oracle, x, d):
+    want = element_codes_by_division(oracle, x, d)
+    got, decided = element_codes_by_bracket(oracle, x, d)
+    bad = decided & (got != want)
+    assert not bad.any(), (f"{bad.sum()} bracket codes differ from the division; first x={x[bad][0]!r} "
+                           f"d={d[bad][0]!r}")
+    return decided.mean()
+
+
+def test_element_brackets_random(oracle):
+    rng = np.random.default_rng(1)
+    n = 2_000_000
+    s = e4m3_values(oracle)[rng.integers(0, 126, n)]
+    g = F(2.0) ** rng.uniform(-40, 20, n).astype(np.float32)
+    d = (s * g).astype(np.float32)
+    x = (rng.standard_normal(n).astype(np.float32) * d * F(3)).astype(np.float32)
+    decided = check_elements(oracle, x, d)
+    assert decided > 0.999  # the division is the rare path
+
+
+@pytest.mark.parametrize("m", E2M1_MIDPOINTS + [6.0, 7.0])
+def test_element_brackets_at_every_midpoint(oracle, m):
+    """x within 64 ulps of m * d, both signs, over every e4m3 scale times
+    random global scales: the operands most likely to break the shortcut."""
+    rng = np.random.default_rng(int(m * 8))
+    s = e4m3_values(oracle)
+    g = F(2.0) ** rng.uniform(-30, 30, 64).astype(np.float32)
+    d = (s[:, None] * g[None, :]).astype(np.float32).ravel()
+    x0 = (F(m) * d).astype(np.float32)
+    k = np.arange(-64, 65, dtype=np.int64)
+    bits = x0.view(np.uint32).astype(np.int64)[:, None] + k[None, :]
+    x = bits.astype(np.uint32).view(np.float32).ravel()
+    dd = np.repeat(d, k.size)
+    x = np.concatenate([x, -x])
+    dd = np.concatenate([dd, dd])
+    check_elements(oracle, x, dd)
+
+
+def test_element_brackets_tiny_and_huge_divisors(oracle):
+    """Divisors at the edges of the shortcut's range, and beyond it."""
+    rng = np.random.default_rng(3)
+    exps = np.array([-149, -140, -127, -126, -125, -124, 120, 124, 125, 126, 127], dtype=np.float64)
+    d = np.repeat((2.0 ** exps * rng.uniform(1, 2, exps.size)).astype(np.float32), 4096)
+    x64 = rng.standard_normal(d.size) * d.astype(np.float64) * 3
+    x = np.clip(x64, -3.4e38, 3.4e38).astype(np.float32)
+    check_elements(oracle, x, d)
+
+
+def scale_codes(oracle, a, g):
+    """(bracket code, decided, code by the two divisions)."""
+    with np.errstate(over="ignore", under="ignore", divide="ignore", invalid="ignore"):
+        rg = F(1) / g
+        t1 = (a * F(1.0 / 6.0)) * rg
+        lo = np.maximum(t1 * LO20, MIN_SCALE)
+        hi = np.maximum(t1 * HI20, MIN_SCALE)
+        chain = np.maximum((a / F(6)) / g, MIN_SCALE)
+    clo, chi = oracle.e4m3_round(lo), oracle.e4m3_round(hi)
+    ok_range = (g >= F(2.0 ** -125)) & (g <= F(2.0 ** 125)) & ((a == 0) | (a >= F(2.0 ** -120)))
+    return clo, (clo == chi) & ok_range, oracle.e4m3_round(chain)
+
+
+def check_scales(oracle, a, g):
+    got, decided, want = scale_codes(oracle, a, g)
+    bad = decided & (got != want)
+    assert not bad.any(), f"{bad.sum()} scale codes differ; first a={a[bad][0]!r} g={g[bad][0]!r}"
+    return decided.mean()
+
+
+def test_scale_brackets_random(oracle):
+    rng = np.random.default_rng(4)
+    n = 2_000_000
+    amax_row = F(2.0) ** rng.uniform(-30, 30, n).astype(np.float32)
+    g = (amax_row / F(2688)).astype(np.float32)
+    a = (amax_row * rng.uniform(0, 1, n).astype(np.float32)).astype(np.float32)
+    a[::97] = 0
+    decided = check_scales(oracle, a, g)
+    assert decided > 0.999
+
+
+def test_scale_brackets_at_every_e4m3_boundary(oracle):
+    """a / 6 / g within 64 ulps of every e4m3 rounding boundary (the midpoint
+    between adjacent codes) and of every code value, for random g."""
+    rng = np.random.default_rng(5)
+    vals = np.concatenate([[0.0], e4m3_values(oracle).astype(np.float64)])
+    mids = (vals[1:] + vals[:-1]) / 2
+    targets = np.concatenate([vals[1:], mids, [448.0 * 1.0625, 2.0 ** -10]])
+    g = (F(2.0) ** rng.uniform(-20, 20, 32)).astype(np.float32)
+    a0 = (targets[:, None] * 6.0 * g[None, :].astype(np.float64)).astype(np.float32).ravel()
+    k = np.arange(-64, 65, dtype=np.int64)
+    a = (a0.view(np.uint32).astype(np.int64)[:, None] + k[None, :]).astype(np.uint32).view(np.float32).ravel()
+    gg = np.repeat(np.tile(g, targets.size), k.size)
+    check_scales(oracle, a, gg)
+
+
+def test_the_brackets_are_needed(oracle):
+    """Taking RN(x * RN(1/d)) without brackets gets some codes wrong on the
+    boundary operands above, and so does a scale taken from t1 alone: the
+    boundary cases are really exercised, and the brackets are what makes the
+    shortcut exact."""
+    s = e4m3_values(oracle)
+    rng = np.random.default_rng(6)
+    g = F(2.0) ** rng.uniform(-30, 30, 64).astype(np.float32)
+    d = (s[:, None] * g[None, :]).astype(np.float32).ravel()
+    wrong = 0
+    for m in E2M1_MIDPOINTS:
+        x0 = (F(m) * d).astype(np.float32)
+        for k in (-2, -1, 0, 1, 2):
+            x = (x0.view(np.uint32).astype(np.int64) + k).astype(np.uint32).view(np.float32)
+            with np.errstate(over="ignore", under="ignore"):
+                q = x * (F(1) / d)
+            wrong += int((oracle.e2m1_round(q) != element_codes_by_division(oracle, x, d)).sum())
+    assert wrong > 0
+
+    vals = e4m3_values(oracle).astype(np.float64)
+    mids = (vals[1:] + vals[:-1]) / 2
+    gg = (F(2.0) ** rng.uniform(-20, 20, 32)).astype(np.float32)
+    a0 = (mids[:, None] * 6.0 * gg[None, :].astype(np.float64)).astype(np.float32).ravel()
+    g2 = np.tile(gg, mids.size)
+    wrong = 0
+    for k in range(-4, 5):
+        a = (a0.view(np.uint32).astype(np.int64) + k).astype(np.uint32).view(np.float32)
+        with np.errstate(over="ignore", under="ignore"):
+            t1 = np.maximum((a * F(1.0 / 6.0)) * (F(1) / g2), MIN_SCALE)
+            chain = np.maximum((a / F(6)) / g2, MIN_SCALE)
+        wrong += int((oracle.e4m3_round(t1) != oracle.e4m3_round(chain)).sum())
+    assert wrong > 0
