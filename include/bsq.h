@@ -138,7 +138,10 @@ bsq_status bsq_dequantize_nvfp4(const uint8_t* packed, const uint8_t* scales_e4m
  * (e2m1 * e4m3) * g in binary32 with one final rounding to yt.
  * values, scales and amax are device arrays of nblocks device pointers
  * (8-byte aligned arrays; the pointed-to blocks may have any alignment).
- * One launch for all blocks; at most 2**32 output items (8 bf16 or 4 fp32). */
+ * One launch for all blocks.  Errors: BSQ_ERR_INVALID_ARG for negative
+ * sizes, null or misaligned arrays/output; BSQ_ERR_UNSUPPORTED for more than
+ * 2**32 output items in all (an item is 8 bf16 or 4 fp32 outputs) or more
+ * than 2**32 outputs in one block.  No blocks, or empty blocks: nothing. */
 bsq_status bsq_dequantize_kv_cache_nvfp4(const uint8_t* const* values, const uint8_t* const* scales,
                                          const float* const* amax, int64_t nblocks, int64_t block_tokens,
                                          int64_t heads, void* y, bsq_dtype yt, bsq_stream_t stream);
