@@ -53,7 +53,8 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the sub-measurements of the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--only", default="", help="run only these sub-measurements (comma list of nvfp4,mxfp8,kv,"
-                    "cache,linear,gemm) and print them, without the main step; for profiling")
+                    "cache,linear,gemm; linear_tensor, linear_row, linear_gu, linear_dq, linear_static pick one row "
+                    "of linear) and print them, without the main step; for profiling")
     ap.add_argument("--gemm-only", default="", help="time only these grouped-GEMM variants (comma list of "
                     "mxfp4_fwd,mxfp4_bwd,nvfp4_fwd,nvfp4_bwd) and print them; for profiling")
     return ap.parse_args()
@@ -226,32 +227,287 @@ def l2_flush(torch, buf):
     buf.max()
 
 
-def oracle_cpu_sample(rows, seconds_target=10.0):
-    """Time the CPU oracle (single thread, as it stands) on `rows` rows of the
-    [8*2048, 7168] workload: quantize + dequantize bf16 + dequantize fp32."""
+# ------------------------------------------------------- CPU oracle baseline -
+#
+# The CPU oracle, as it stands (plain scalar C called through ctypes), timed on
+# the host cores.  ctypes releases the GIL for the length of each C call, so
+# host threads that each run the oracle on their own slice of rows run in
+# parallel; nothing in the oracle is changed or tuned for this.  Every row of
+# the path gets two figures: one thread, and one thread per core of
+# os.sched_getaffinity.  Samples are whole rows (or cache blocks) of the same
+# workloads, sized to a fraction of a second per figure; the rate is bytes (or
+# FLOPs) per second, so a sample and the full tensor share the unit.
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _run_parts(fn, parts, threads):
+    """Wall seconds to run fn(part) for every part on `threads` host threads."""
+    from concurrent.futures import ThreadPoolExecutor
+    t0 = time.perf_counter()
+    if threads <= 1:
+        for part in parts:
+            fn(part)
+    else:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(fn, parts))
+    return time.perf_counter() - t0
+
+
+def _split_rows(a, n):
+    """n contiguous row slices of a (views; the oracle needs no copy)."""
+    import numpy as np
+    edges = np.linspace(0, a.shape[0], n + 1).astype(int)
+    return [a[edges[i]:edges[i + 1]] for i in range(n) if edges[i + 1] > edges[i]]
+
+
+class OracleCase:
+    """One row of the path for the CPU oracle: make(rows) builds a seeded input
+    of `rows` rows (untimed), run(part) processes a row slice of it,
+    bytes_per_row is the row's algorithmic bytes (as on the GPU)."""
+
+    def __init__(self, make, run, bytes_per_row, full_rows, split=None):
+        self.make, self.run, self.bytes_per_row, self.full_rows = make, run, bytes_per_row, full_rows
+        self.split = split or _split_rows
+
+
+def time_oracle_case(case, cores, seconds=0.4, probe_rows=8):
+    """Single-thread and all-core rates of one case, in GB/s, on samples sized
+    to about `seconds` each (never more rows than the full workload)."""
+    probe = case.make(probe_rows)
+    t = max(_run_parts(case.run, [probe], 1), 1e-4)
+    rows1 = int(max(probe_rows, min(case.full_rows, probe_rows * seconds / t)))
+    x1 = case.make(rows1)
+    t1 = _run_parts(case.run, [x1], 1)
+    del x1
+    rows_n = int(max(rows1, min(case.full_rows, rows1 * cores)))
+    xn = case.make(rows_n)
+    parts = case.split(xn, cores)
+    tn = _run_parts(case.run, parts, cores)
+    b1, bn = rows1 * case.bytes_per_row, rows_n * case.bytes_per_row
+    return {"single_thread": {"GB/s": round(b1 / t1 / 1e9, 4), "rows": rows1, "s": round(t1, 3)},
+            "all_cores": {"GB/s": round(bn / tn / 1e9, 4), "rows": rows_n, "s": round(tn, 3), "threads": len(parts)},
+            "full_rows": case.full_rows}
+
+
+def mx_round_trip_case():
+    """The bench step's workload: MXFP4 quantize + dequantize to bf16 and fp32,
+    rows of 7168 from the [8*2048, 7168] expert weights."""
+    import oracle
+    from fp8_microscaling_quantization_b200 import synth
+
+    def make(rows):
+        return synth.expert_weights(E=1, N=rows, K=K, zero_blocks=min(4, rows * K // 32), seed=20260002).reshape(rows, K)
+
+    def run(x):
+        pk, sc = oracle.quantize_mxfp4(x)
+        oracle.dequantize_mxfp4(pk, sc, out_dtype=oracle.BF16)
+        oracle.dequantize_mxfp4(pk, sc, out_dtype=oracle.F32)
+
+    q, d1, d2 = mx_bytes()
+    return OracleCase(make, run, (q + d1 + d2) // (E * N), E * N)
+
+
+def oracle_cases():
+    """The CPU oracle's counterpart of every sub-measurement, keyed as in the
+    GPU output: {(section, row): OracleCase}."""
     import numpy as np
     import oracle
     from fp8_microscaling_quantization_b200 import synth
-    w = synth.expert_weights(E=1, N=rows, K=K, zero_blocks=4, seed=20260002).reshape(rows, K)
-    t0 = time.perf_counter()
-    p, s = oracle.quantize_mxfp4(w)
-    oracle.dequantize_mxfp4(p, s, out_dtype=oracle.BF16)
-    oracle.dequantize_mxfp4(p, s, out_dtype=oracle.F32)
-    dt = time.perf_counter() - t0
-    n = rows * K
-    nbytes = (2 * n + n // 2 + n // 32) + (n // 2 + n // 32 + 2 * n) + (n // 2 + n // 32 + 4 * n)
-    return nbytes, dt
+    cases = {}
+
+    # NVFP4 [256, 2048], per-row scale: quantize; dequantize to bf16
+    Kn = 2048
+    nb = 2 * Kn + Kn // 2 + Kn // 16 + 4
+    cases[("nvfp4_256x2048", "quantize")] = OracleCase(
+        lambda r: synth.nvfp4_matrix(rows=r, cols=Kn, seed=20260001), lambda x: oracle.quantize_nvfp4(x), nb, 256)
+
+    def make_nv_q(rows, cols=Kn, seed=20260001):
+        # dequantize inputs: random packed codes, finite e4m3 scales, row scales
+        rng = np.random.default_rng(seed)
+        return (rng.integers(0, 256, (rows, cols // 2), dtype=np.uint8),
+                rng.integers(0, 0x7F, (rows, cols // 16), dtype=np.uint8),
+                (rng.random(rows) * 1e-3).astype(np.float32))
+
+    def split3(t, n):
+        pk, sc, g = t
+        return list(zip(_split_rows(pk, n), _split_rows(sc, n), _split_rows(g, n)))
+
+    cases[("nvfp4_256x2048", "dequantize_bf16")] = OracleCase(
+        make_nv_q, lambda t: oracle.dequantize_nvfp4(*t, out_dtype=oracle.BF16), nb, 256, split3)
+
+    # MXFP8 on the [8, 2048, 7168] expert weights
+    def make_w(rows):
+        return synth.expert_weights(E=1, N=rows, K=K, zero_blocks=min(4, rows * K // 32), seed=20260006).reshape(rows, K)
+
+    def split2(t, n):
+        return list(zip(_split_rows(t[0], n), _split_rows(t[1], n)))
+
+    cases[("mxfp8_expert_weights_8x2048x7168", "quantize")] = OracleCase(
+        make_w, lambda x: oracle.quantize_mxfp8(x), 2 * K + K + K // 32, E * N)
+    def make_mx8_codes(rows):
+        rng = np.random.default_rng(20260006)
+        c = rng.integers(0, 0x7F, (rows, K), dtype=np.uint8) | (rng.integers(0, 2, (rows, K), dtype=np.uint8) << 7)
+        return (c, rng.integers(100, 130, (rows, K // 32), dtype=np.uint8))
+
+    cases[("mxfp8_expert_weights_8x2048x7168", "dequantize_bf16")] = OracleCase(
+        make_mx8_codes, lambda t: oracle.dequantize_mxfp8(*t, out_dtype=oracle.BF16), K + K // 32 + 2 * K, E * N,
+        split2)
+
+    # KV cache: a "row" is one block of 64 tokens x 8 heads x 128
+    bt, hd = 64, 8
+    rows_kv = bt * hd
+
+    def make_kv(nblk):
+        rng = np.random.default_rng(20260007)
+        vals = [rng.integers(0, 256, (rows_kv, 64), dtype=np.uint8) for _ in range(nblk)]
+        scs = [rng.integers(0, 0x7E, (rows_kv, 8), dtype=np.uint8) for _ in range(nblk)]
+        am = (rng.random(nblk) * 100).astype(np.float32)
+        return (vals, scs, am)
+
+    def split_kv(t, n):
+        vals, scs, am = t
+        edges = np.linspace(0, len(vals), n + 1).astype(int)
+        return [(vals[a:b], scs[a:b], am[a:b]) for a, b in zip(edges[:-1], edges[1:]) if b > a]
+
+    nkv = rows_kv * 128
+    cases[("kv_cache_nvfp4_1024x64x8x128", "dequantize_bf16")] = OracleCase(
+        make_kv, lambda t: oracle.dequantize_kv_cache_nvfp4(t[0], t[1], t[2], bt, hd), nkv // 2 + nkv // 16 + 4 + 2 * nkv,
+        1024, split_kv)
+
+    # quantize_cache: a row is one [C] vector of the [B, T, C] activations
+    for name, fmt, blk, (Bc, Tc, C) in (
+            ("fp8_b32_4x8192x512", 0, 32, (4, 8192, 512)), ("mxfp4_b32_4x8192x128", 1, 32, (4, 8192, 128)),
+            ("nvfp4_b16_4x2048x512", 2, 16, (4, 2048, 512)), ("fp8_b32_4x2048x520", 0, 32, (4, 2048, 520)),
+            ("mxfp4_b32_4x2048x520", 1, 32, (4, 2048, 520)), ("nvfp4_b16_4x2048x520", 2, 16, (4, 2048, 520))):
+        cases[("quantize_cache", name)] = OracleCase(
+            (lambda C: lambda r: synth.cache_acts(B=1, T=r, C=C, seed=20260003)[0].reshape(r, C))(C),
+            (lambda fmt, blk: lambda x: oracle.quantize_cache(x, fmt, blk))(fmt, blk), 4 * C, Bc * Tc)
+    cases[("quantize_cache", "ste_backward_copy_4x8192x512")] = OracleCase(
+        lambda r: synth.cache_acts(B=1, T=r, C=512, seed=20260003)[1].reshape(r, 512),
+        lambda g: oracle.quantize_cache_backward(g), 4 * 512, 4 * 8192)
+
+    # [7168, 18432] linear weight
+    Kl = 18432
+    nrow = 2 * Kl + Kl // 2 + Kl // 16
+
+    def make_lin(r):
+        return synth.linear_weight(out=r, inp=Kl, seed=20260004)
+
+    sec = "nvfp4_linear_7168x18432"
+    # per-tensor: each thread quantizes its own slice with that slice's tensor
+    # scale (the same work per element as one tensor scale over all rows)
+    cases[(sec, "modelopt_tensor_scale")] = OracleCase(make_lin, lambda x: oracle.quantize_nvfp4_tensor(x),
+                                                       nrow + 2 * Kl, 7168)
+    cases[(sec, "per_row_scale")] = OracleCase(make_lin, lambda x: oracle.quantize_nvfp4(x), nrow + 4, 7168)
+
+    def make_gu(r):
+        x = make_lin(r)
+        return (x, np.full(r, 1e-5, np.float32))
+
+    cases[(sec, "gate_up_given_row_scales_14336x18432")] = OracleCase(
+        make_gu, lambda t: oracle.quantize_nvfp4(t[0], row_scale=t[1]), nrow + 8, 14336, split2)
+    cases[(sec, "dequantize_bf16")] = OracleCase(
+        lambda r: make_nv_q(r, Kl, 20260004), lambda t: oracle.dequantize_nvfp4(*t, out_dtype=oracle.BF16),
+        Kl // 2 + Kl // 16 + 4 + 2 * Kl, 7168, split3)
+
+    def make_static(r):
+        x = make_lin(r)
+        xf = synth.bf16_bits_to_f32(x)
+        bam = np.abs(xf).reshape(r, -1, 16).max(axis=2).astype(np.float32)
+        return (x, bam, float(np.abs(xf).max()))
+
+    def split_static(t, n):
+        return [(a, b, t[2]) for a, b in zip(_split_rows(t[0], n), _split_rows(t[1], n))]
+
+    cases[(sec, "static_two_level_fake_quant")] = OracleCase(
+        make_static, lambda t: oracle.fake_quantize_nvfp4_static(*t), 2 * Kl + 4 * (Kl // 16) + 2 * Kl, 7168,
+        split_static)
+    return cases
+
+
+def time_oracle_gemm(cores, offs):
+    """The grouped GEMM's CPU reference (the oracle's binary32 dequantization of
+    each expert, then a float64 library matmul), timed on one expert with a
+    sample of rows and extrapolated linearly to the full problem: 32 expert
+    dequantizations plus T rows of products.  The matmul uses the BLAS threads
+    of numpy (one, then `cores`)."""
+    import numpy as np
+    import oracle
+    from threadpoolctl import threadpool_limits
+    from fp8_microscaling_quantization_b200 import synth
+    T, Kd, Nd, Ed = 16384, 7168, 2048, 32
+    rows = 256
+    rng = np.random.default_rng(20260005)
+    w = synth.to_bf16_bits((rng.standard_normal((Nd, Kd), dtype=np.float32) * np.float32(0.02)))
+    pk, sc = oracle.quantize_mxfp4(w)
+    a = synth.to_bf16_bits(rng.standard_normal((rows, Kd), dtype=np.float32))
+    del w
+    out = {}
+    for label, threads in (("single_thread", 1), ("all_cores", cores)):
+        with threadpool_limits(limits=threads):
+            t0 = time.perf_counter()
+            W = oracle.dequant_expert_f32(oracle.FMT_MXFP4, pk, sc).astype(np.float64)
+            t_dq = time.perf_counter() - t0
+            A = oracle.bf16_to_f32(a).astype(np.float64)
+            t0 = time.perf_counter()
+            _ = A @ W.T
+            t_mm = time.perf_counter() - t0
+        t_full = Ed * t_dq + T / rows * t_mm
+        out[label] = {"TFLOP/s": round(2.0 * T * Nd * Kd / t_full / 1e12, 6), "s_full_extrapolated": round(t_full, 2),
+                      "threads": threads}
+    out["sample"] = (f"MXFP4 forward: one expert [2048, 7168] dequantized by the oracle, then {rows} rows of the "
+                     f"float64 product; extrapolated to 32 experts and T=16384 (extrapolated)")
+    return out
+
+
+def run_cpu_oracle_rows(cores):
+    """CPU oracle figures for every sub-measurement: {section: {row: {...}}}."""
+    res = {}
+    for (sec, row), case in oracle_cases().items():
+        try:
+            t0 = time.perf_counter()
+            res.setdefault(sec, {})[row] = time_oracle_case(case, cores)
+            res[sec][row]["wall_s"] = round(time.perf_counter() - t0, 2)
+        except Exception as ex:  # report, never hide
+            res.setdefault(sec, {})[row] = {"unavailable": f"{type(ex).__name__}: {ex}"}
+    try:
+        res["grouped_gemm"] = {"mxfp4_fwd": time_oracle_gemm(cores, None)}
+    except Exception as ex:
+        res["grouped_gemm"] = {"unavailable": f"{type(ex).__name__}: {ex}"}
+    return res
 
 
 def run_cpu_baseline():
-    rows = 128
-    nbytes, dt = oracle_cpu_sample(rows)
-    # scale the sample to about 10 s of CPU work
-    rows2 = int(max(128, min(8192, rows * 10.0 / max(dt, 1e-3))))
-    nbytes, dt = oracle_cpu_sample(rows2)
-    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{rows2} rows x 7168 of the MXFP4 expert-weight workload (quantize + dequantize bf16 + "
-                      f"dequantize fp32), single-threaded C oracle, {dt:.1f} s"}
+    """The bench step's workload on the CPU oracle: all cores (the reported
+    value) and one thread."""
+    cores = host_cores()
+    r = time_oracle_case(mx_round_trip_case(), cores, seconds=2.0)
+    mt, st = r["all_cores"], r["single_thread"]
+    return {"value": mt["GB/s"], "unit": "GB/s", "cores": mt["threads"], "kind": "oracle",
+            "single_thread": {"value": st["GB/s"], "cores": 1, "rows": st["rows"], "s": st["s"]},
+            "sample": f"{mt['rows']} rows x 7168 of the MXFP4 expert-weight workload (quantize + dequantize bf16 + "
+                      f"dequantize fp32), C oracle on {mt['threads']} host threads, {mt['s']} s; single thread: "
+                      f"{st['rows']} rows, {st['s']} s"}
+
+
+def merge_oracle_rows(extra, oracle_rows):
+    """Put each CPU-oracle figure beside its GPU row as "oracle_cpu"."""
+    for sec, rows in oracle_rows.items():
+        dst = extra.setdefault(sec, {})
+        if not isinstance(dst, dict):
+            continue
+        if sec == "grouped_gemm":
+            dst["oracle_cpu"] = rows
+            continue
+        for row, fig in rows.items():
+            ent = dst.setdefault(row, {})
+            if isinstance(ent, dict):
+                ent["oracle_cpu"] = fig
 
 
 # --------------------------------------------------------------- reference --
@@ -261,25 +517,29 @@ def run_reference(args):
     if rank != 0:
         return
     steps, warmup = max(1, args.steps), max(0, args.warmup)
-    rows = 64
+    cores = host_cores()
+    case = mx_round_trip_case()
+    rows = 256 * cores  # 256 rows per host thread per step
+    x = case.make(rows)
+    parts = case.split(x, cores)
     for _ in range(warmup):
-        oracle_cpu_sample(rows)
-    tot_b, tot_t = 0, 0.0
+        _run_parts(case.run, parts, cores)
+    tot_t, done = 0.0, 0
     t_start = time.perf_counter()
     for _ in range(steps):
-        b, t = oracle_cpu_sample(rows)
-        tot_b += b
-        tot_t += t
+        tot_t += _run_parts(case.run, parts, cores)
+        done += 1
         if time.perf_counter() - t_start > 150:
             break
-    val = tot_b / tot_t / 1e9
+    val = done * rows * case.bytes_per_row / tot_t / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": args.gpus,
-            "steps": steps, "warmup": warmup, "ms_per_step": round(tot_t / max(1, steps) * 1e3, 3),
+            "steps": done, "warmup": warmup, "ms_per_step": round(tot_t / done * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": "mxfp4_expert_weights_round_trip", "shape": [E, N, K],
                        "sample_rows_per_step": rows},
-            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{rows} rows x 7168 per step (quantize + dequantize bf16 + fp32)"},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": len(parts), "kind": "oracle",
+                             "sample": f"{rows} rows x 7168 per step (quantize + dequantize bf16 + fp32) on "
+                                       f"{len(parts)} host threads"},
             "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -419,6 +679,8 @@ def main():
             line["cpu_baseline"] = {"unavailable": f"{type(ex).__name__}: {ex}"}
     if not args.no_extra and world == 1:
         line["extra"] = run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, set())
+        if rank == 0 and not args.no_cpu:
+            merge_oracle_rows(line["extra"], run_cpu_oracle_rows(host_cores()))
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -591,12 +853,14 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
         res["note"] = "L2 flushed before every launch (tensors of 8-34 MB)"
         out["quantize_cache"] = res
 
-    if want("linear"):
+    linear_rows = ("tensor", "row", "gu", "dq", "static")
+    want_linear = [r for r in linear_rows if want("linear") or f"linear_{r}" in only]
+    if want_linear:
         g = torch.Generator(device=dev)
         g.manual_seed(20260004)
         x = synth.linear_weight_torch(7168, 18432, generator=g, device=dev)
         up = synth.linear_weight_torch(7168, 18432, generator=g, device=dev)
-        cat = torch.cat([x, up], 0)
+        cat = torch.cat([x, up], 0) if "gu" in want_linear else None
         del up
         n = x.numel()
         p = torch.empty((7168, 18432 // 2), dtype=torch.uint8, device=dev)
@@ -617,20 +881,28 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
         bam = x.view(-1, 16).abs().amax(dim=1).float()
         gam = x.abs().amax().float().reshape(1)
         nb_st = 2 * n + 4 * (n // 16) + 2 * n
-        out["nvfp4_linear_7168x18432"] = {
-            "modelopt_tensor_scale": rec(timed(lambda: bsq.bsq_quantize_nvfp4_tensor(
+        lin = {}
+        if "tensor" in want_linear:
+            lin["modelopt_tensor_scale"] = rec(timed(lambda: bsq.bsq_quantize_nvfp4_tensor(
                 x, packed=p, scales=s, tensor_scale=t, scratch=scratch), 10, False), nb_tensor,
-                "nvfp4_tensor_amax_pass", "nvfp4_tensor_quant_pass"),
-            "per_row_scale": rec(timed(lambda: bsq.bsq_quantize_nvfp4(x, packed=p, scales=s, row_scale_out=r),
-                                       10, False), nb_row, "nvfp4_per_row"),
-            "gate_up_given_row_scales_14336x18432": rec(timed(lambda: bsq.bsq_quantize_nvfp4(
+                "nvfp4_tensor_amax_pass", "nvfp4_tensor_quant_pass")
+        if "row" in want_linear:
+            lin["per_row_scale"] = rec(timed(lambda: bsq.bsq_quantize_nvfp4(x, packed=p, scales=s, row_scale_out=r),
+                                             10, False), nb_row, "nvfp4_per_row")
+        if "gu" in want_linear:
+            lin["gate_up_given_row_scales_14336x18432"] = rec(timed(lambda: bsq.bsq_quantize_nvfp4(
                 cat, row_scale_in=rc, packed=pc, scales=sc, row_scale_out=rco), 10, False), nb_gu,
-                "nvfp4_gate_up_given_row_scales"),
-            "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_nvfp4(p, s, r, y=y), 10, False), nb_dq,
-                                   "nvfp4_dequant_bf16"),
-            "static_two_level_fake_quant": rec(timed(lambda: bsq.bsq_fake_quantize_nvfp4_static(x, bam, gam, y=y),
-                                                     10, False), nb_st, "nvfp4_static_fake_quant"),
-            "note": "inputs larger than L2; per-tensor counts two reads of the input"}
+                "nvfp4_gate_up_given_row_scales")
+        if "dq" in want_linear:
+            bsq.bsq_quantize_nvfp4(x, packed=p, scales=s, row_scale_out=r)
+            lin["dequantize_bf16"] = rec(timed(lambda: bsq.bsq_dequantize_nvfp4(p, s, r, y=y), 10, False), nb_dq,
+                                         "nvfp4_dequant_bf16")
+        if "static" in want_linear:
+            lin["static_two_level_fake_quant"] = rec(timed(
+                lambda: bsq.bsq_fake_quantize_nvfp4_static(x, bam, gam, y=y), 10, False), nb_st,
+                "nvfp4_static_fake_quant")
+        lin["note"] = "inputs larger than L2; per-tensor counts two reads of the input"
+        out["nvfp4_linear_7168x18432"] = lin
         del x, cat, y
 
     if want("gemm"):

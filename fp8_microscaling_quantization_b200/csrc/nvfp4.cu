@@ -263,6 +263,8 @@ static __device__ __align__(256) float g_noalloc_partials[kNoAllocMaxPartials];
 
 // Device address of g_noalloc_partials, looked up once per device with that
 // device current (in host code the array's name is only a host-side handle).
+// The address is cached for the life of the process; a device reset, which
+// tears down the context the module was loaded in, leaves it stale.
 static float* noalloc_partials_ptr(bsq_status* st) {
     static std::mutex mu;
     static float* ptrs[64] = {nullptr};

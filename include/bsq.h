@@ -109,7 +109,10 @@ bsq_status bsq_quantize_nvfp4_tensor(const void* x, bsq_dtype xt, int64_t rows, 
  *     BSQ_ERR_UNSUPPORTED.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept for the rest of the
+ *     process: after cudaDeviceReset (or anything else that destroys and
+ *     re-creates the device's primary context) it no longer names the array,
+ *     so do not call this entry point on that device again in the process.
  *   - All calls share the one array: calls whose kernels overlap on the GPU
  *     (concurrent streams) race and give wrong results.  Serialise them.
  *     Nothing needs clearing between calls. */

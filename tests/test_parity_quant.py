@@ -36,7 +36,10 @@ def edge_bf16_values():
 
 # ---------------------------------------------------------------- NVFP4 -----
 
-@pytest.mark.parametrize("rows,K", [(256, 2048), (37, 272), (5, 16), (129, 4096), (3, 40000), (1, 32768)])
+# K > 65536 takes the two-kernel form (row amax pass, then the flat quantize
+# reading the computed row scales); the rest run the one-CTA-per-row kernel.
+@pytest.mark.parametrize("rows,K", [(256, 2048), (37, 272), (5, 16), (129, 4096), (3, 40000), (1, 32768),
+                                    (1, 65536), (3, 65552), (2, 131072)])
 def test_nvfp4_rowamax_bf16(B, S, oracle, rows, K):
     x = S.nvfp4_matrix(rows=rows, cols=K, seed=1000 + rows + K)
     p, s, g = B.bsq_quantize_nvfp4(dev_bf16(x))
@@ -51,9 +54,11 @@ def test_nvfp4_rowamax_bf16(B, S, oracle, rows, K):
     assert_bits_equal(host_bits(y32), oracle.dequantize_nvfp4(op, os_, og, out_dtype=oracle.F32), "dequant fp32")
 
 
-def test_nvfp4_rowamax_fp32_input(B, S, oracle):
-    rng = np.random.default_rng(5)
-    x = (rng.standard_normal((64, 1024)) * np.exp(rng.uniform(-20, 20, (64, 1)))).astype(np.float32)
+@pytest.mark.parametrize("rows,K", [(64, 1024), (3, 65552)])
+def test_nvfp4_rowamax_fp32_input(B, S, oracle, rows, K):
+    rng = np.random.default_rng(5 + K)
+    x = (rng.standard_normal((rows, K)) * np.exp(rng.uniform(-20, 20, (rows, 1)))).astype(np.float32)
+    x[0, 7] *= 30.0  # an outlier that sets the row maximum
     p, s, g = B.bsq_quantize_nvfp4(dev(x))
     op, os_, og = oracle.quantize_nvfp4(x)
     assert_bits_equal(host_bits(g), og, "row scale")
@@ -163,6 +168,21 @@ def test_nvfp4_full_size_linear_weight(B, S, oracle):
     rs = torch.cat([t.expand(x.shape[0]), tu.expand(up.shape[0])]).contiguous()
     pc, sc, gc = B.bsq_quantize_nvfp4(cat, row_scale_in=rs)
     torch.cuda.synchronize()
+    tu_ref = np.float32(np.abs(f32_of(up)).max()) / np.float32(2688.0)
+    assert host_bits(tu)[0] == tu_ref
+    # both halves of the concatenation against the oracle, each row with its
+    # half's tensor scale
+    urows = sample_rows(up.shape[0], 48, 2)
+    cat_rows = np.concatenate([rows, x.shape[0] + urows])
+    csub = np.ascontiguousarray(np.concatenate([x[rows], up[urows]]))
+    g_rows = np.concatenate([np.full(rows.size, t_ref, np.float32), np.full(urows.size, tu_ref, np.float32)])
+    op, os_, og = oracle.quantize_nvfp4(csub, row_scale=g_rows)
+    assert_bits_equal(host_bits(gc)[cat_rows], og, "gate/up row scales (sampled rows)")
+    assert_bits_equal(host_bits(pc)[cat_rows], op, "gate/up packed (sampled rows)")
+    assert_bits_equal(host_bits(sc)[cat_rows], os_, "gate/up e4m3 scales (sampled rows)")
+    # and the up half's own per-tensor quantization on its sampled rows
+    assert_bits_equal(host_bits(pu)[urows], op[rows.size:], "up tensor packed (sampled rows)")
+    assert_bits_equal(host_bits(su)[urows], os_[rows.size:], "up tensor scales (sampled rows)")
     assert torch.equal(pc, torch.cat([p, pu])) and torch.equal(sc, torch.cat([s, su]))
 
 

@@ -49,6 +49,22 @@ def test_noalloc_matches_scratch_entry_point_twice(B):
         assert_bits_equal(got[0], want[0], "packed")
 
 
+def test_noalloc_same_shape_lower_amax(B):
+    """Two calls of one shape back to back, the second on a tensor whose
+    maximum is far lower: every partial maximum the second call reads must be
+    its own, or the first call's larger amax would leak into its tensor scale."""
+    from fp8_microscaling_quantization_b200 import synth
+    big = dev_bf16(synth.linear_weight(out=1024, inp=4096, seed=904))
+    low = (big.float() * 0.01).to(torch.bfloat16)
+    for x in (big, low):
+        want, got = _both(B, x)
+        assert_bits_equal(got[2], want[2], "tensor scale")
+        assert_bits_equal(got[1], want[1], "e4m3 scales")
+        assert_bits_equal(got[0], want[0], "packed")
+    amax_low = low.float().abs().max().item()
+    assert got[2].view(np.float32)[0] == np.float32(amax_low) / np.float32(2688.0)
+
+
 def test_noalloc_fp32_input_and_empty(B):
     rng = np.random.default_rng(903)
     x = torch.from_numpy(rng.standard_normal((300, 512)).astype(np.float32)).cuda()
