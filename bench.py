@@ -56,7 +56,7 @@ def parse_args():
                     "cache,linear,gemm; linear_tensor, linear_row, linear_gu, linear_dq, linear_static pick one row "
                     "of linear) and print them, without the main step; for profiling")
     ap.add_argument("--gemm-only", default="", help="time only these grouped-GEMM variants (comma list of "
-                    "mxfp4_fwd,mxfp4_bwd,nvfp4_fwd,nvfp4_bwd) and print them; for profiling")
+                    "mxfp4_fwd,mxfp4_bwd,nvfp4_fwd,nvfp4_bwd,skew) and print them; for profiling")
     return ap.parse_args()
 
 
@@ -923,7 +923,7 @@ def bench_gemm(torch, bsq, synth, dev, stream, peaks, peak_kind, variants=None, 
     x = torch.randn((T, Kd), generator=g, device=dev).to(torch.bfloat16)
     go = torch.randn((T, Nd), generator=g, device=dev).to(torch.bfloat16)
     w = (torch.randn((Ed, Nd, Kd), generator=g, device=dev) * 0.02).to(torch.bfloat16)
-    want_mx = not variants or any(v.startswith("mxfp4") for v in variants)
+    want_mx = not variants or any(v.startswith("mxfp4") or v == "skew" for v in variants)
     want_nv = not variants or any(v.startswith("nvfp4") for v in variants)
     mx_p, mx_s = bsq.bsq_quantize_mxfp4(w) if want_mx else (None, None)
     nv_p, nv_s, nv_r = bsq.bsq_quantize_nvfp4(w) if want_nv else (None, None, None)
@@ -952,6 +952,29 @@ def bench_gemm(torch, bsq, synth, dev, stream, peaks, peak_kind, variants=None, 
             res[f"{fmt_name}_{dname}"] = {"us": round(ms * 1e3, 1), "TFLOP/s": round(tf, 1),
                                           "frac_bf16": round(tf / peak, 4),
                                           "traffic": traffic_from_profiles(f"gemm_{fmt_name}_{dname}")}
+    # routing skews (MXFP4 forward, same weights and activations): how the
+    # 16-token padding of short experts and the tile dealing hold up
+    if not variants or "skew" in variants:
+        skew = {}
+        for kind in ("uniform", "zipf", "hot", "tiny"):
+            o_np = synth.skew_offs(np.random.default_rng(20260008), kind, T, Ed)
+            o = torch.from_numpy(o_np).to(dev)
+            fn = lambda: bsq.bsq_grouped_mm_fp4(bsq.Format.MXFP4, bsq.Direction.FWD, x, mx_p, mx_s, None, o,
+                                                out=out_f, err=err)
+            t = Timer(torch, stream)
+            for _ in range(warm):
+                fn()
+            for _ in range(iters):
+                t.run("k", fn)
+            torch.cuda.synchronize()
+            ms = t.avg_ms("k")
+            tf = flops / (ms * 1e-3) / 1e12
+            cnt = np.diff(np.concatenate([[0], o_np]))
+            skew[kind] = {"us": round(ms * 1e3, 1), "TFLOP/s": round(tf, 1), "frac_bf16": round(tf / peak, 4),
+                          "max_expert_tokens": int(cnt.max()), "experts_under_17_tokens": int((cnt < 17).sum())}
+        skew["note"] = "MXFP4 forward, T=16384 K=7168 N=2048 E=32; routing: uniform, Zipf(1.1), one expert with " \
+                       "half the tokens, half the experts with 1-16 tokens"
+        res["routing_skew_mxfp4_fwd"] = skew
     res["err_word"] = int(err.item())
     res["peak"] = f"{peak} TFLOP/s bf16 dense ({peak_kind}, burst)"
     return res

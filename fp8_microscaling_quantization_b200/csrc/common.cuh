@@ -203,6 +203,228 @@ __device__ __forceinline__ uint2 nv_quant_block(const float v[16], float g, floa
     return make_uint2(e2m1x8_of_quotient(v, d), e2m1x8_of_quotient(v + 8, d));
 }
 
+// ---- lean NVFP4 block: shared reciprocal table, brackets on the reciprocal --
+//
+// Per-CTA table of RN(1/s) over the e4m3 scale codes (index = code, positive
+// finite codes 1..126; the rest 0), filled once per CTA.
+__device__ __forceinline__ void fill_inv_e4m3(float* tab) {
+    for (int c = threadIdx.x; c < 128; c += blockDim.x)
+        tab[c] = (c >= 1 && c <= 126) ? __frcp_rn(e4m3_decode((uint32_t)c)) : 0.0f;
+}
+
+// max(|a|, |b|) of each bf16 lane of two bf16x2 words (the sign of the result
+// is the XOR of the signs; only the magnitude is used).
+__device__ __forceinline__ uint32_t bf16x2_maxabs(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// 16 elements of one NVFP4 block as loaded (bf16: two uint4, fp32: four
+// float4), widened to binary32 on use.
+template <typename T> struct Raw16;
+// 16 bytes from a 32-bit shared-memory address.
+__device__ __forceinline__ uint4 lds128(uint32_t saddr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
+    return v;
+}
+
+template <> struct Raw16<uint16_t> {
+    uint4 a, b;
+    __device__ __forceinline__ void load(const uint16_t* p) {
+        a = reinterpret_cast<const uint4*>(p)[0];
+        b = reinterpret_cast<const uint4*>(p)[1];
+    }
+    __device__ __forceinline__ void load_smem(uint32_t saddr) {
+        a = lds128(saddr);
+        b = lds128(saddr + 16);
+    }
+    // block amax, exact (bf16 -> binary32 widening is exact)
+    __device__ __forceinline__ float amax() const {
+        const uint32_t m = bf16x2_maxabs(bf16x2_maxabs(bf16x2_maxabs(a.x, a.y), bf16x2_maxabs(a.z, a.w)),
+                                         bf16x2_maxabs(bf16x2_maxabs(b.x, b.y), bf16x2_maxabs(b.z, b.w)));
+        return fmaxf(fabsf(bf16_lo(m)), fabsf(bf16_hi(m)));
+    }
+    __device__ __forceinline__ void half(int h, float v[8]) const {
+        const uint4 w = h ? b : a;
+        v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+        v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+    }
+};
+template <> struct Raw16<float> {
+    float4 q[4];
+    __device__ __forceinline__ void load(const float* p) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) q[i] = reinterpret_cast<const float4*>(p)[i];
+    }
+    __device__ __forceinline__ void load_smem(uint32_t saddr) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 w = lds128(saddr + 16 * i);
+            q[i] = make_float4(__uint_as_float(w.x), __uint_as_float(w.y), __uint_as_float(w.z), __uint_as_float(w.w));
+        }
+    }
+    __device__ __forceinline__ float amax() const {
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            m = fmaxf(fmaxf(m, fmaxf(fabsf(q[i].x), fabsf(q[i].y))), fmaxf(fabsf(q[i].z), fabsf(q[i].w)));
+        return m;
+    }
+    __device__ __forceinline__ void half(int h, float v[8]) const {
+        const float4 c = q[2 * h], d = q[2 * h + 1];
+        v[0] = c.x; v[1] = c.y; v[2] = c.z; v[3] = c.w; v[4] = d.x; v[5] = d.y; v[6] = d.z; v[7] = d.w;
+    }
+};
+
+// Two binary32 products at once (packed f32x2 multiply of sm_100a; each lane
+// rounds to nearest even exactly as a scalar multiply does).
+__device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 A, B, D;\n\t"
+        "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+        "mul.rn.f32x2 D, A, B;\n\t"
+        "mov.b64 {%0, %1}, D;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// Asynchronous 16-byte global -> shared copies (cp.async, L2 only), grouped
+// per thread; a thread waits for its own groups with cp_async_wait.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The block's codes by the plain rule (IEEE division where the brackets
+// cannot decide); kept out of line, it runs for a tiny fraction of blocks.
+template <typename T>
+__device__ __noinline__ uint2 nv_block_codes_slow(Raw16<T> raw, float g, uint32_t s) {
+    const float d = __fmul_rn(e4m3_decode(s), g);
+    float v[8];
+    raw.half(0, v);
+    const uint32_t c0 = e2m1x8_of_quotient(v, d);
+    raw.half(1, v);
+    return make_uint2(c0, e2m1x8_of_quotient(v, d));
+}
+
+// The division-free part of nv_block_codes below: false when the brackets
+// disagree or r is out of range (the caller then takes the plain rule, away
+// from its hot loop).  g != 0.
+
+// The codes of a block whose brackets disagree (nv_block_codes_fast returned
+// false), bit-exact and still without a division.  blk holds the block's 16
+// elements, s its scale code, rg = nv_recip_or_zero(g).  An element whose two
+// bracket codes differ has exactly one e2m1 rounding boundary b between them
+// (0.25, 0.75, 1.25, 1.75, 2.5, 3.5 or 5; the brackets are far narrower than
+// the gaps), and |x| lies within 2**-20 of b * d, d = RN(float(s) * g), so
+// e = fma(-b, d, |x|) is the exact difference.  With hu half an ulp of b and
+// hd half an ulp of the float below b (hu / 2 for b = 0.25, a power of two):
+// RN(|x| / d) > b iff e > hu * d, < b iff e < -hd * d, else it equals b, an
+// e2m1 tie that rounds to the even code.  (b's significand is even, so the
+// roundings of b + hu and b - hd are b itself.)  If r is out of range the
+// plain rule is taken.
+// Element i of a block held in shared memory at saddr, as binary32.
+template <typename T>
+__device__ __forceinline__ float elem_smem(uint32_t saddr, int i);
+template <>
+__device__ __forceinline__ float elem_smem<uint16_t>(uint32_t saddr, int i) {
+    uint32_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(saddr + 2u * (uint32_t)i));
+    return __uint_as_float(v << 16);
+}
+template <>
+__device__ __forceinline__ float elem_smem<float>(uint32_t saddr, int i) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(saddr + 4u * (uint32_t)i));
+    return v;
+}
+
+// Settles the nibbles of clo (the lower bracket's codes of the 8 elements at
+// shared address half) where the upper bracket's codes differ (set bits of
+// diff), by the fma test above.
+// Per lower magnitude code k = 0..6 of a straddle: the e2m1 rounding boundary
+// b above it, and the half ulps hu (of b) and hd (of the float below b).
+struct NvBound {
+    float b, hu, hd, pad;
+};
+__device__ __forceinline__ void fill_nv_bounds(NvBound* t) {
+    if (threadIdx.x < 8) {
+        const int k = threadIdx.x;
+        // e2m1 magnitudes: k < 4: k / 2; then 2, 3, 4, 6; b is the midpoint to the next
+        const float b = (k < 4) ? 0.25f + 0.5f * (float)k : (k == 4 ? 2.5f : (k == 5 ? 3.5f : (k == 6 ? 5.0f : 6.0f)));
+        const int eb = floor_log2_exact(b);
+        t[k].b = b;
+        t[k].hu = exp2_int(eb - 24);
+        t[k].hd = (k == 0) ? exp2_int(eb - 25) : exp2_int(eb - 24);
+        t[k].pad = 0.0f;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t nv_settle_straddles(uint32_t clo, uint32_t diff, uint32_t half, float d,
+                                                        const NvBound* bounds) {
+    while (diff) {
+        const int sh = (__ffs(diff) - 1) & ~3;  // 4 * nibble index
+        diff &= ~(0xFu << sh);
+        const uint32_t cl = (clo >> sh) & 0xFu;
+        const uint32_t k = cl & 7u;  // the lower magnitude code (lo <= hi in magnitude)
+        const NvBound bd = bounds[k];
+        const float x = elem_smem<T>(half, sh >> 2);
+        const float e = __fmaf_rn(-bd.b, d, fabsf(x));
+        const uint32_t mag = (e > __fmul_rn(bd.hu, d)) ? k + 1u : ((e < -__fmul_rn(bd.hd, d)) ? k : ((k + 1u) & ~1u));
+        clo = (clo & ~(0xFu << sh)) | (((cl & 8u) | mag) << sh);
+    }
+    return clo;
+}
+
+
+// The division-free codes of one block (the hot path of the NVFP4 quantize
+// kernels): brackets on r = RN(RN(1/s) * rg), and the rare straddled element
+// settled by the fma test.  raw holds the block's 16 elements, blk the shared
+// address of the same elements (read only for a straddled element), s the
+// scale code, g != 0 and rg = nv_recip_or_zero(g).  Returns false only when r
+// is out of range; the caller then takes the plain rule (nv_block_codes_slow).
+template <typename T>
+__device__ __forceinline__ bool nv_block_codes_fast(const Raw16<T>& raw, uint32_t blk, uint32_t s, float g, float rg,
+                                                    const float* inv_tab, const NvBound* bounds, uint2* codes) {
+    const float r = __fmul_rn(inv_tab[s], rg);
+    if (!(r >= 2.3509887e-38f /* 2**-125 */ && r <= 4.2535296e37f /* 2**125 */)) return false;
+    const float2 rlo = make_float2(__fmul_rn(r, 0.99999952f), __fmul_rn(r, 0.99999952f));  // 1 - 2**-21
+    const float2 rhi = make_float2(__fmul_rn(r, 1.00000048f), __fmul_rn(r, 1.00000048f));  // 1 + 2**-21
+    uint32_t clo[2], chi[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float v[8], lo[8], hi[8];
+        raw.half(h, v);
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            const float2 l = mul_f32x2(make_float2(v[j], v[j + 1]), rlo);
+            const float2 u = mul_f32x2(make_float2(v[j], v[j + 1]), rhi);
+            lo[j] = l.x; lo[j + 1] = l.y;
+            hi[j] = u.x; hi[j + 1] = u.y;
+        }
+        clo[h] = e2m1x8_encode_hw(lo);
+        chi[h] = e2m1x8_encode_hw(hi);
+    }
+    const uint32_t d0 = clo[0] ^ chi[0], d1 = clo[1] ^ chi[1];
+    if (d0 | d1) {  // rare: a bracket straddles an e2m1 rounding boundary
+        const float d = __fmul_rn(e4m3x2_decode_hw(s).x, g);  // RN(float(s) * g); s is a positive code
+        if (d0) clo[0] = nv_settle_straddles<T>(clo[0], d0, blk, d, bounds);
+        if (d1) clo[1] = nv_settle_straddles<T>(clo[1], d1, blk + 8u * (uint32_t)sizeof(T), d, bounds);
+    }
+    *codes = make_uint2(clo[0], clo[1]);
+    return true;
+}
+
 // 16 consecutive elements (32-byte aligned for bf16).  Plain (L1-cached)
 // loads: the second half of every line a warp touches is then an L1 hit.
 __device__ __forceinline__ void load16(const uint16_t* p, float v[16]) {

@@ -81,7 +81,7 @@ constexpr uint32_t kWStage = WM * BK * 2;       // 16 KiB dequantized weights
 constexpr uint32_t kXBoxBytes = XBOX * BK * 2;  // 8 KiB
 constexpr int kMaxExperts = 1024;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint64_t kWaitNs = 1000000000ull;  // default limit of a pipeline wait, and of every drain wait
 constexpr int kPrefetch = 4;  // k-steps of packed weights in flight per producer thread
 
 // Shared-memory plan of a CTA group of CG CTAs (1, or a pair with
@@ -120,6 +120,7 @@ struct Args {
     const int32_t* offs;
     uint16_t* out;
     uint32_t* err;
+    uint64_t wait_ns;  // limit of each pipeline wait (kWaitNs unless BSQ_GMM_WAIT_NS says otherwise)
     int E, T, N, K;
 };
 
@@ -163,18 +164,27 @@ __device__ __forceinline__ Shared carve(uint8_t* raw) {
 }
 
 // Bounded wait that also gives up as soon as another role has aborted.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Shared& sh, uint32_t* err) {
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const Shared& sh, const Args& a) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
+    uint32_t* err = a.err;
     while (!mbar_try_wait(bar, parity)) {
         if (*sh.abort) return false;
-        if (globaltimer_ns() - t0 > kWaitNs) {
+        if (globaltimer_ns() - t0 > a.wait_ns) {
             *sh.abort = 1;
             atomicOr(err, (uint32_t)BSQ_DEVERR_TIMEOUT);
             return false;
         }
     }
     return true;
+}
+
+// The same for all 32 lanes of a warp, with one outcome for the whole warp:
+// it gives up if any lane's wait did, so the warp stays converged for the
+// warp-collective instructions (__syncwarp, tcgen05.ld) that follow.
+__device__ __forceinline__ bool wait_bar_warp(uint64_t* bar, uint32_t parity, const Shared& sh, const Args& a) {
+    const bool ok = wait_bar(bar, parity, sh, a);
+    return __all_sync(0xffffffffu, ok);
 }
 
 // f0 is the first feature of the group's tile (CTA r of a pair owns
@@ -429,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
         for (int t = group; t < num_tiles; t += ngroups, ++tile_iter) {
             const Tile ti = decode_tile<CG>(t, f_tiles, E, sh);
             const int acc = tile_iter % P::NACC;
-            if (!wait_bar(&sh.acc_full[acc], (tile_iter / P::NACC) & 1, sh, args.err)) break;
+            if (!wait_bar_warp(&sh.acc_full[acc], (tile_iter / P::NACC) & 1, sh, args)) break;
             tc_fence_after();
             const int f = ti.f0 + WM * (int)rank + q * 32 + lane;
             float gf = 1.0f;
@@ -506,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                         }
                     }
                     const int s = i % P::STAGES;
-                    if (!wait_bar(&sh.empty[s], ((i / P::STAGES) & 1) ^ 1, sh, args.err)) {
+                    if (!wait_bar_warp(&sh.empty[s], ((i / P::STAGES) & 1) ^ 1, sh, args)) {
                         ok = false;
                     } else {
                         store_unit<DIR>(v, st_base + s * P::kStage, dq);
@@ -532,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                 const int nbox0 = (h0 + XBOX - 1) / XBOX, nbox1 = (h1 + XBOX - 1) / XBOX;
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
                     const int s = it % P::STAGES;
-                    if (!wait_bar(&sh.empty[s], ((it / P::STAGES) & 1) ^ 1, sh, args.err)) {
+                    if (!wait_bar(&sh.empty[s], ((it / P::STAGES) & 1) ^ 1, sh, args)) {
                         ok = false;
                         break;
                     }
@@ -582,12 +592,12 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                 const uint32_t idesc0 = idesc_bf16_ab(WM * CG, n0, DIR == BSQ_BWD ? 1u : 0u, 0u);
                 const uint32_t idesc1 = idesc_bf16_ab(WM * CG, n1 ? n1 : 16u, DIR == BSQ_BWD ? 1u : 0u, 0u);
                 const int acc = tile_iter % P::NACC;
-                if (!wait_bar(&sh.acc_empty[acc], ((tile_iter / P::NACC) & 1) ^ 1, sh, args.err)) break;
+                if (!wait_bar(&sh.acc_empty[acc], ((tile_iter / P::NACC) & 1) ^ 1, sh, args)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * TN);
                 for (int ks = 0; ks < k_steps; ++ks, ++it) {
                     const int s = it % P::STAGES;
-                    if (!wait_bar(&sh.full[s], (it / P::STAGES) & 1, sh, args.err)) {
+                    if (!wait_bar(&sh.full[s], (it / P::STAGES) & 1, sh, args)) {
                         ok = false;
                         break;
                     }
@@ -753,6 +763,14 @@ BSQ_API bsq_status bsq_grouped_mm_fp4(bsq_format fmt, bsq_dir dir, const void* a
     args.offs = offs;
     args.out = (uint16_t*)out;
     args.err = err;
+    // BSQ_GMM_WAIT_NS (a positive integer, in ns) shortens the limit of each
+    // pipeline wait; tests use it to make the waits run out on purpose
+    args.wait_ns = gmm::kWaitNs;
+    if (const char* w = getenv("BSQ_GMM_WAIT_NS")) {
+        char* end = nullptr;
+        const unsigned long long v = strtoull(w, &end, 10);
+        if (end != w && *end == '\0' && v > 0) args.wait_ns = v;
+    }
     args.E = E;
     args.T = (int)T;
     args.N = (int)N;

@@ -153,14 +153,248 @@ __global__ void __launch_bounds__(kThreads) nv_flat_quant_kernel(const T* __rest
     }
 }
 
+// ------------------------------------------- rows staged in shared memory
+//
+// One CTA per row (persistent over the rows blockIdx.x + i * gridDim.x).
+// Thread t owns the 16-element blocks t, t + nt, ... (at most kStgMaxBpt) of
+// every row: it copies them into shared memory itself with cp.async, S - 1
+// rows ahead, so the HBM stream runs while earlier rows are computed, and it
+// reads back only its own blocks, so stages are reused without waiting for
+// the other threads.  A first sweep takes the blocks' amaxes; MODE 2 reduces
+// the row amax across the CTA (the kernel's only per-row barrier; per-warp
+// slots alternate by row parity).  A second sweep forms the codes by the
+// division-free brackets.
+//
+// An element whose brackets disagree is settled in place by an exact fma
+// test (nv_block_codes_fast), no division.  With a scale tied to the data (a
+// row or tensor amax / 2688) a few percent of the blocks hold an element whose
+// quotient lands on an e2m1 rounding boundary (an element with the same
+// significand as the amax, for instance), so that path is kept to a few
+// instructions: it runs on one lane of a warp.
+// MODE 0 takes g from g_in, MODE 1 the tensor scale from the partial maxima,
+// MODE 2 the row's own amax / 2688.  NT is the launch's maximum thread count,
+// MINB the CTAs per SM the register budget is sized for.
+constexpr int kStgMaxThreads = 512, kStgMaxBpt = 4;
+
+template <typename T, int MODE, int S, int NT, int MINB>
+__global__ void __launch_bounds__(NT, MINB)
+    nv_row_staged_kernel(const T* __restrict__ x, int64_t rows, int K, const float* __restrict__ g_in,
+                         const float* __restrict__ partial, int npartial, uint8_t* __restrict__ packed,
+                         uint8_t* __restrict__ scales, float* __restrict__ g_out) {
+    extern __shared__ __align__(128) uint8_t stage_mem[];
+    __shared__ float red[2][NT / 32];
+    __shared__ float inv_tab[128];
+    __shared__ NvBound bounds[8];
+    constexpr int kCopies = (int)sizeof(T);  // 16-byte copies per block: 2 (bf16) or 4 (fp32)
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+    const int bpr = K / 16;
+    const uint32_t stage_bytes = ((uint32_t)K * (uint32_t)sizeof(T) + 127u) & ~127u;
+    fill_inv_e4m3(inv_tab);
+    fill_nv_bounds(bounds);
+    float g_t = 0.0f, rg_t = 0.0f;
+    if (MODE == 1) {
+        float m = 0.0f;
+        for (int i = tid; i < npartial; i += nt) m = fmaxf(m, partial[i]);
+        m = group_max<32>(m);
+        if (lane == 0) red[0][warp] = m;
+    }
+    __syncthreads();
+    if (MODE == 1) {
+        float m = lane < nw ? red[0][lane] : 0.0f;
+        m = group_max<32>(m);
+        g_t = __fdiv_rn(m, kNvGlobalDiv);
+        rg_t = nv_recip_or_zero(g_t);
+        if (blockIdx.x == 0 && tid == 0) g_out[0] = g_t;
+        __syncthreads();  // red[0] is reused by the rows below
+    }
+    const int64_t first = blockIdx.x, step = gridDim.x;
+    const int64_t my_rows = (first < rows) ? (rows - 1 - first) / step + 1 : 0;
+    // this thread's blocks: byte offsets within a row (32-bit), and how many
+    constexpr uint32_t kBlkBytes = 16u * (uint32_t)sizeof(T);
+    const uint32_t smem0 = (uint32_t)__cvta_generic_to_shared(stage_mem);
+    const int myb = (bpr > tid) ? min(kStgMaxBpt, (bpr - 1 - tid) / nt + 1) : 0;
+    auto issue = [&](int64_t i) {
+        if (i < my_rows) {
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(x + (first + i * step) * (int64_t)K);
+            const uint32_t dst = smem0 + (uint32_t)(i % S) * stage_bytes;
+#pragma unroll
+            for (int j = 0; j < kStgMaxBpt; ++j) {
+                if (j < myb) {
+                    const uint32_t off = (uint32_t)(tid + j * nt) * kBlkBytes;
+#pragma unroll
+                    for (int c = 0; c < kCopies; ++c)
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + off + 16u * c),
+                                     "l"(src + off + 16u * c)
+                                     : "memory");
+                }
+            }
+        }
+        cp_async_commit();  // one group per row, empty past the last row
+    };
+#pragma unroll
+    for (int i = 0; i < S - 1; ++i) issue(i);
+    for (int64_t i = 0; i < my_rows; ++i) {
+        const int64_t r = first + i * step;
+        issue(i + S - 1);        // into the stage of row i - 1, which this thread has finished
+        cp_async_wait<S - 1>();  // this thread's copies of row i have landed
+        const uint32_t xs = smem0 + (uint32_t)(i % S) * stage_bytes;  // shared address of row i
+        float am[kStgMaxBpt];
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kStgMaxBpt; ++j) {
+            am[j] = 0.0f;
+            if (j < myb) {
+                Raw16<T> raw;
+                raw.load_smem(xs + (uint32_t)(tid + j * nt) * kBlkBytes);
+                am[j] = raw.amax();
+                m = fmaxf(m, am[j]);
+            }
+        }
+        float g;
+        if (MODE == 2) {
+            m = group_max<32>(m);
+            if (lane == 0) red[i & 1][warp] = m;
+            __syncthreads();
+            float mm = lane < nw ? red[i & 1][lane] : 0.0f;
+            mm = group_max<32>(mm);
+            g = __fdiv_rn(mm, kNvGlobalDiv);
+        } else if (MODE == 0) {
+            g = g_in[r];
+        } else {
+            g = g_t;
+        }
+        if (MODE != 1 && tid == 0) g_out[r] = g;
+        const float rg = (MODE == 1) ? rg_t : nv_recip_or_zero(g);
+        uint8_t* prow = packed + r * (int64_t)(K / 2);
+        uint8_t* srow = scales + r * (int64_t)bpr;
+        uint32_t redo_self = 0u;
+#pragma unroll
+        for (int j = 0; j < kStgMaxBpt; ++j) {
+            if (j < myb) {
+                const int b = tid + j * nt;
+                const uint32_t blk = xs + (uint32_t)b * kBlkBytes;
+                uint32_t sb = 0u;
+                uint2 pk = make_uint2(0u, 0u);
+                if (g != 0.0f) {
+                    Raw16<T> raw;
+                    raw.load_smem(blk);
+                    sb = nv_scale_code(am[j], g, rg);
+                    if (!nv_block_codes_fast<T>(raw, blk, sb, g, rg, inv_tab, bounds, &pk)) redo_self |= 1u << j;
+                }
+                reinterpret_cast<uint2*>(prow)[b] = pk;
+                srow[b] = (uint8_t)sb;
+            }
+        }
+        while (redo_self) {  // r out of range (g near the ends of the binary32 range)
+            const int j = __ffs(redo_self) - 1;
+            redo_self &= redo_self - 1u;
+            const int b = tid + j * nt;
+            Raw16<T> raw;
+            raw.load_smem(xs + (uint32_t)b * kBlkBytes);
+            reinterpret_cast<uint2*>(prow)[b] = nv_block_codes_slow<T>(raw, g, nv_scale_code(am[j], g, rg));
+        }
+    }
+    cp_async_wait<0>();
+}
+
 }  // namespace bsq
 
 using namespace bsq;
+
+// Staged-row launch plan for rows of K elements of T: threads per CTA (a
+// multiple of 32, at most kStgMaxBpt blocks each), stages of the ring and the
+// register-budget variant: up to 384 threads run three CTAs of two stages per
+// SM (56 registers a thread) when their stages fit, otherwise two CTAs of
+// three (or two) stages (64 registers).  nt = 0: the row does not fit.
+struct StagedPlan {
+    int nt = 0, stages = 0;
+    bool three = false;
+    size_t smem = 0;
+};
+
+template <typename T>
+static StagedPlan staged_plan(int64_t K) {
+    StagedPlan p;
+    const int64_t bpr = K / 16;
+    const int64_t row_bytes = K * (int64_t)sizeof(T);
+    if (bpr < 1 || bpr > (int64_t)kStgMaxThreads * kStgMaxBpt || row_bytes > 100 * 1024) return p;
+    const int64_t stage_bytes = (row_bytes + 127) / 128 * 128;
+    const int bpt = (int)((bpr + kStgMaxThreads - 1) / kStgMaxThreads);
+    const int64_t per = (bpr + bpt - 1) / bpt;
+    p.nt = (int)((per + 31) / 32 * 32);
+    // per CTA: the stages, under 1 KiB of static shared memory and 1 KiB the
+    // hardware reserves, against the 228 KiB of an SM
+    if (p.nt <= 384 && 3 * (2 * stage_bytes + 4 * 1024) <= 228 * 1024) {
+        p.three = true;
+        p.stages = 2;
+    } else {
+        p.stages = (3 * stage_bytes <= 110 * 1024) ? 3 : 2;
+    }
+    p.smem = (size_t)(p.stages * stage_bytes);
+    return p;
+}
+
+template <typename T, int MODE, int S, int NT, int MINB>
+static bsq_status launch_staged_v(const StagedPlan& p, const T* x, int64_t rows, int64_t K, const float* g_in,
+                                  const float* partial, int npartial, uint8_t* packed, uint8_t* scales, float* g_out,
+                                  cudaStream_t st, const char* fn) {
+    static std::mutex mu;
+    static size_t opted[64] = {0};
+    auto kern = nv_row_staged_kernel<T, MODE, S, NT, MINB>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (opted[dev] < p.smem) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+            if (e != cudaSuccess) return fail(BSQ_ERR_CUDA, "%s: shared-memory opt-in failed (%s)", fn, cudaGetErrorString(e));
+            opted[dev] = p.smem;
+        }
+    }
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, p.nt, p.smem) != cudaSuccess || per_sm < 1) {
+        cudaGetLastError();
+        per_sm = 1;
+    }
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(rows, (int64_t)sm_count() * per_sm));
+    kern<<<grid, p.nt, p.smem, st>>>(x, rows, (int)K, g_in, partial, npartial, packed, scales, g_out);
+    return check_launch(fn);
+}
+
+template <typename T, int MODE>
+static bsq_status launch_staged(const StagedPlan& p, const T* x, int64_t rows, int64_t K, const float* g_in,
+                                const float* partial, int npartial, uint8_t* packed, uint8_t* scales, float* g_out,
+                                cudaStream_t st, const char* fn) {
+    if (p.three)
+        return launch_staged_v<T, MODE, 2, 384, 3>(p, x, rows, K, g_in, partial, npartial, packed, scales, g_out, st, fn);
+    if (p.stages == 3)
+        return launch_staged_v<T, MODE, 3, kStgMaxThreads, 2>(p, x, rows, K, g_in, partial, npartial, packed, scales,
+                                                               g_out, st, fn);
+    return launch_staged_v<T, MODE, 2, kStgMaxThreads, 2>(p, x, rows, K, g_in, partial, npartial, packed, scales,
+                                                           g_out, st, fn);
+}
+
+// Second pass of the ModelOpt layout: quantize with the tensor scale reduced
+// from the P partial maxima (staged rows where they fit, else flat blocks).
+template <typename T>
+static bsq_status launch_tensor_quant(const T* x, int64_t rows, int64_t K, const float* partial, int P,
+                                      uint8_t* packed, uint8_t* scales, float* tensor_scale_out, cudaStream_t st,
+                                      const char* fn) {
+    const StagedPlan sp = staged_plan<T>(K);
+    if (sp.nt) return launch_staged<T, 1>(sp, x, rows, K, nullptr, partial, P, packed, scales, tensor_scale_out, st, fn);
+    const int64_t nblocks = rows * (K / 16);
+    launch_fit<nv_flat_quant_kernel<T, 1, 2>>(nblocks, 2, st, x, nblocks, make_fastdiv((uint32_t)(K / 16)),
+                                              (const float*)nullptr, partial, P, packed, scales, tensor_scale_out);
+    return check_launch(fn);
+}
 
 template <typename T>
 static bsq_status launch_nv_rowamax(const T* x, int64_t rows, int64_t K, uint8_t* packed, uint8_t* scales,
                                     float* g_out, cudaStream_t st) {
     const int64_t cpr = K / 8;
+    const StagedPlan sp = staged_plan<T>(K);
+    if (sp.nt) return launch_staged<T, 2>(sp, x, rows, K, nullptr, nullptr, 0, packed, scales, g_out, st,
+                                          "bsq_quantize_nvfp4");
     if (K <= 65536) {
         static_assert(kRowThreads == kThreads, "row kernel launched with the common block size");
         launch_fit_ctas<nv_rowamax_quant_kernel<T>>(rows, st, x, rows, K, packed, scales, g_out);
@@ -187,6 +421,17 @@ BSQ_API bsq_status bsq_quantize_nvfp4(const void* x, bsq_dtype xt, int64_t rows,
     if (!aligned(x, 16) || !aligned(packed, 8)) return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4: misaligned pointer");
     cudaStream_t st = (cudaStream_t)stream;
     if (row_scale_in) {
+        if (xt == BSQ_BF16) {
+            const StagedPlan sp = staged_plan<uint16_t>(K);
+            if (sp.nt)
+                return launch_staged<uint16_t, 0>(sp, (const uint16_t*)x, rows, K, row_scale_in, nullptr, 0, packed,
+                                                  scales_e4m3, row_scale_out, st, "bsq_quantize_nvfp4");
+        } else {
+            const StagedPlan sp = staged_plan<float>(K);
+            if (sp.nt)
+                return launch_staged<float, 0>(sp, (const float*)x, rows, K, row_scale_in, nullptr, 0, packed,
+                                               scales_e4m3, row_scale_out, st, "bsq_quantize_nvfp4");
+        }
         const int64_t nblocks = rows * (K / 16);
         const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
         if (xt == BSQ_BF16)
@@ -230,23 +475,18 @@ BSQ_API bsq_status bsq_quantize_nvfp4_tensor(const void* x, bsq_dtype xt, int64_
     if (scratch_bytes < (size_t)P * sizeof(float))
         return fail(BSQ_ERR_INVALID_ARG, "bsq_quantize_nvfp4_tensor: scratch of %zu bytes, need %zu", scratch_bytes,
                     (size_t)P * sizeof(float));
-    const int64_t nchunks = rows * (K / 8), nblocks = rows * (K / 16);
+    const int64_t nchunks = rows * (K / 8);
     float* partial = (float*)scratch;
-    const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
     if (xt == BSQ_BF16) {
         amax_partial_kernel<uint16_t, 4><<<P, kThreads, 0, st>>>((const uint16_t*)x, nchunks, partial);
         BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor"));
-        launch_fit<nv_flat_quant_kernel<uint16_t, 1, 2>>(nblocks, 2, st, (const uint16_t*)x, nblocks, bpr,
-                                                         (const float*)nullptr, (const float*)partial, P, packed,
-                                                         scales_e4m3, tensor_scale_out);
-    } else {
-        amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
-        BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor"));
-        launch_fit<nv_flat_quant_kernel<float, 1, 2>>(nblocks, 2, st, (const float*)x, nblocks, bpr,
-                                                      (const float*)nullptr, (const float*)partial, P, packed,
-                                                      scales_e4m3, tensor_scale_out);
+        return launch_tensor_quant((const uint16_t*)x, rows, K, partial, P, packed, scales_e4m3, tensor_scale_out, st,
+                                   "bsq_quantize_nvfp4_tensor");
     }
-    return check_launch("bsq_quantize_nvfp4_tensor");
+    amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
+    BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor"));
+    return launch_tensor_quant((const float*)x, rows, K, partial, P, packed, scales_e4m3, tensor_scale_out, st,
+                               "bsq_quantize_nvfp4_tensor");
 }
 
 // ----------------------------------------------- no-allocation variant ----
@@ -313,21 +553,17 @@ BSQ_API bsq_status bsq_quantize_nvfp4_tensor_noalloc(const void* x, bsq_dtype xt
     bsq_status status;
     float* partial = noalloc_partials_ptr(&status);
     if (!partial) return status;
-    const int64_t nchunks = rows * (K / 8), nblocks = rows * (K / 16);
-    const FastDiv bpr = make_fastdiv((uint32_t)(K / 16));
+    const int64_t nchunks = rows * (K / 8);
     if (xt == BSQ_BF16) {
         amax_partial_kernel<uint16_t, 4><<<P, kThreads, 0, st>>>((const uint16_t*)x, nchunks, partial);
         BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
-        launch_fit<nv_flat_quant_kernel<uint16_t, 1, 2>>(nblocks, 2, st, (const uint16_t*)x, nblocks, bpr,
-                                                         (const float*)nullptr, (const float*)partial, P, packed,
-                                                         scales_e4m3, tensor_scale_out);
-    } else {
-        amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
-        BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
-        launch_fit<nv_flat_quant_kernel<float, 1, 2>>(nblocks, 2, st, (const float*)x, nblocks, bpr,
-                                                      (const float*)nullptr, (const float*)partial, P, packed,
-                                                      scales_e4m3, tensor_scale_out);
+        return launch_tensor_quant((const uint16_t*)x, rows, K, partial, P, packed, scales_e4m3, tensor_scale_out, st,
+                                   "bsq_quantize_nvfp4_tensor_noalloc");
     }
-    return check_launch("bsq_quantize_nvfp4_tensor_noalloc");
+    amax_partial_kernel<float, 4><<<P, kThreads, 0, st>>>((const float*)x, nchunks, partial);
+    BSQ_TRY(check_launch("bsq_quantize_nvfp4_tensor_noalloc"));
+    return launch_tensor_quant((const float*)x, rows, K, partial, P, packed, scales_e4m3, tensor_scale_out, st,
+                               "bsq_quantize_nvfp4_tensor_noalloc");
 }
+
 

@@ -106,6 +106,38 @@ def zipf_offs(rng, tokens: int, E: int, s: float = 1.1) -> np.ndarray:
     return np.cumsum(counts).astype(np.int32)
 
 
+def skew_offs(rng, kind: str, tokens: int, E: int) -> np.ndarray:
+    """int32 cumulative token counts for a routing skew:
+    "uniform"  every expert the same share (the remainder to the first ones);
+    "zipf"     zipf_offs above (Zipf 1.1, one expert emptied);
+    "hot"      one expert (seeded) holds half the tokens, the rest are spread
+               uniformly at random over the others;
+    "tiny"     half the experts get 1-16 tokens each (seeded), the other half
+               share the rest evenly."""
+    if kind == "zipf":
+        return zipf_offs(rng, tokens, E)
+    counts = np.zeros(E, np.int64)
+    if kind == "uniform":
+        counts[:] = tokens // E
+        counts[: tokens - counts.sum()] += 1
+    elif kind == "hot":
+        h = int(rng.integers(0, E))
+        counts[h] = tokens // 2
+        rest = [e for e in range(E) if e != h]
+        counts[rest] = rng.multinomial(tokens - counts[h], np.full(E - 1, 1.0 / (E - 1)))
+    elif kind == "tiny":
+        small = rng.permutation(E)[: E // 2]
+        counts[small] = rng.integers(1, 17, small.size)
+        big = np.setdiff1d(np.arange(E), small)
+        left = tokens - counts.sum()
+        counts[big] = left // big.size
+        counts[big[: left - counts[big].sum()]] += 1
+    else:
+        raise ValueError(f"unknown routing skew {kind!r}")
+    assert counts.sum() == tokens
+    return np.cumsum(counts).astype(np.int32)
+
+
 def moe_problem(T=16384, K=7168, N=2048, E=32, seed=None, with_weights=True):
     """Returns dict(x bf16 [T,K], offs int32 [E], w bf16 [E,N,K] or None, grad_out bf16 [T,N])."""
     rng = _rng(seed, 5)

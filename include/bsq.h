@@ -61,7 +61,7 @@ typedef enum { BSQ_FWD = 0, BSQ_BWD = 1 } bsq_dir;
 
 /* Bits of the device error word written by bsq_grouped_mm_fp4. */
 #define BSQ_DEVERR_BAD_OFFS 1u  /* offs not non-decreasing, negative, or offs[E-1] > T */
-#define BSQ_DEVERR_TIMEOUT 2u   /* a pipeline wait gave up after its time limit (about 1 s) */
+#define BSQ_DEVERR_TIMEOUT 2u   /* a pipeline wait gave up after its time limit (1 s, or BSQ_GMM_WAIT_NS) */
 
 const char* bsq_status_string(bsq_status s);
 const char* bsq_last_error(void);
@@ -246,6 +246,12 @@ bsq_status bsq_quantize_cache_backward(const void* grad_out, void* grad_in, bsq_
  *   err         device uint32 word; the caller zeroes it before the call and
  *               reads it after synchronising: BSQ_DEVERR_* bits.  With a bad
  *               offs the output is undefined.
+ * Every wait between the kernel's pipeline roles gives up after 1 s: the
+ * kernel then sets BSQ_DEVERR_TIMEOUT, lets its outstanding loads and MMAs
+ * finish, frees its tensor memory and returns (the output is undefined, the
+ * context stays usable).  The environment variable BSQ_GMM_WAIT_NS, read at
+ * every call, sets another limit in nanoseconds (a test hook: a limit of a
+ * few ns makes the waits run out).
  * Rows at or past offs[E-1] are written as zero.  Requirements: the output
  * width (N for BSQ_FWD, K for BSQ_BWD) a multiple of 128 and K, N multiples
  * of 64; E <= 1024; a, packed, out and row_scale 16-byte aligned.  Other

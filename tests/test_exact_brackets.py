@@ -40,6 +40,36 @@ def element_codes_by_bracket(oracle, x, d):
     return clo, (clo == chi) & in_range
 
 
+def element_codes_by_scaled_reciprocal(oracle, x, s, g):
+    """The kernels' element shortcut for d = RN(s * g), s an e4m3 value:
+    r = RN(RN(1/s) * RN(1/g)) (RN(1/s) from a table over the e4m3 codes, RN(1/g)
+    once per row), then the brackets are put on r, not on the quotient:
+    lo = RN(x * RN(r * (1 - 2**-21))), hi = RN(x * RN(r * (1 + 2**-21))).
+    r is within 4 roundings of 1/d (those of RN(s*g), RN(1/s), RN(1/g) and the
+    product) and each bracket adds two, so lo and hi lie within 6 * 2**-24 of
+    x/d * (1 -+ 2**-21): they enclose RN(x/d), which is within 2**-24 of x/d,
+    whenever r is normal.  (code, decided)."""
+    with np.errstate(over="ignore", under="ignore", invalid="ignore", divide="ignore"):
+        inv_s = F(1) / s
+        rg = F(1) / g
+        r = inv_s * rg
+        lo, hi = x * (r * LO21), x * (r * HI21)
+    clo, chi = oracle.e2m1_round(lo), oracle.e2m1_round(hi)
+    in_range = (r >= F(2.0 ** -125)) & (r <= F(2.0 ** 125)) & (g >= F(2.0 ** -125)) & (g <= F(2.0 ** 125))
+    return clo, (clo == chi) & in_range
+
+
+def check_elements_scaled(oracle, x, s, g):
+    with np.errstate(over="ignore", under="ignore"):
+        d = (s * g).astype(np.float32)
+    want = element_codes_by_division(oracle, x, d)
+    got, decided = element_codes_by_scaled_reciprocal(oracle, x, s, g)
+    bad = decided & (got != want)
+    assert not bad.any(), (f"{bad.sum()} scaled-reciprocal codes differ from the division; first x={x[bad][0]!r} "
+                           f"s={s[bad][0]!r} g={g[bad][0]!r}")
+    return decided.mean()
+
+
 def element_codes_by_division(oracle, x, d):
     with np.errstate(over="ignore", under="ignore", divide="ignore", invalid="ignore"):
         return oracle.e2m1_round(x / d)
@@ -176,3 +206,150 @@ def test_the_brackets_are_needed(oracle):
             chain = np.maximum((a / F(6)) / g2, MIN_SCALE)
         wrong += int((oracle.e4m3_round(t1) != oracle.e4m3_round(chain)).sum())
     assert wrong > 0
+
+
+def test_scaled_reciprocal_random(oracle):
+    rng = np.random.default_rng(7)
+    n = 2_000_000
+    s = e4m3_values(oracle)[rng.integers(0, 126, n)]
+    g = F(2.0) ** rng.uniform(-40, 20, n).astype(np.float32)
+    d = (s * g).astype(np.float32)
+    x = (rng.standard_normal(n).astype(np.float32) * d * F(3)).astype(np.float32)
+    decided = check_elements_scaled(oracle, x, s, g)
+    assert decided > 0.999
+
+
+@pytest.mark.parametrize("m", E2M1_MIDPOINTS + [6.0, 7.0])
+def test_scaled_reciprocal_at_every_midpoint(oracle, m):
+    """x within 64 ulps of m * RN(s * g), both signs, over every e4m3 scale s
+    and random g (including g whose product with s is not exact)."""
+    rng = np.random.default_rng(int(m * 16) + 1)
+    sv = e4m3_values(oracle)
+    g = (F(2.0) ** rng.uniform(-30, 30, 64).astype(np.float32) * rng.uniform(1, 2, 64).astype(np.float32))
+    ss = np.repeat(sv, g.size)
+    gg = np.tile(g.astype(np.float32), sv.size)
+    d = (ss * gg).astype(np.float32)
+    x0 = (F(m) * d).astype(np.float32)
+    k = np.arange(-64, 65, dtype=np.int64)
+    x = (x0.view(np.uint32).astype(np.int64)[:, None] + k[None, :]).astype(np.uint32).view(np.float32).ravel()
+    ss, gg = np.repeat(ss, k.size), np.repeat(gg, k.size)
+    x = np.concatenate([x, -x])
+    check_elements_scaled(oracle, x, np.concatenate([ss, ss]), np.concatenate([gg, gg]))
+
+
+def test_scaled_reciprocal_at_the_range_edges(oracle):
+    """g near the ends of the range where RN(1/g) is normal, and s*g near the
+    ends of the range where r is normal (the shortcut must then stand aside)."""
+    rng = np.random.default_rng(8)
+    sv = e4m3_values(oracle)
+    exps = np.array([-134, -130, -126, -125, -124, -117, 110, 116, 117, 124, 125, 126], dtype=np.float64)
+    g = (2.0 ** exps * rng.uniform(1, 2, exps.size)).astype(np.float32)
+    ss = np.repeat(sv, g.size * 64)
+    gg = np.tile(np.repeat(g, 64), sv.size)
+    with np.errstate(over="ignore", under="ignore"):
+        d = (ss * gg).astype(np.float64)
+    x = np.clip(rng.standard_normal(ss.size) * d * 3, -3.4e38, 3.4e38).astype(np.float32)
+    check_elements_scaled(oracle, x, ss, gg)
+
+
+# ---- power-of-two block scale without the division -------------------------
+#
+# The cache fake-quant's scale is pow2ceil(max(RN(a / M), 2**-126)) for
+# M = 448 (fp8) or 6 (mxfp4).  q = RN(a * RN(1/M)) is within two roundings of
+# a / M and RN(a / M) within one, and pow2ceil is monotone, so when the two
+# brackets RN(q * (1 -+ 2**-21)) have the same power-of-two ceiling, that is
+# RN(a / M)'s; the kernels divide only when they differ or q < 2**-125.
+
+def pow2_by_bracket(oracle, a, M):
+    with np.errstate(over="ignore", under="ignore"):
+        q = a * (F(1) / F(M))
+        lo, hi = q * LO21, q * HI21
+    plo, phi = oracle.pow2_ceil(np.maximum(lo, F(2.0 ** -126))), oracle.pow2_ceil(np.maximum(hi, F(2.0 ** -126)))
+    return plo, (plo == phi) & (q >= F(2.0 ** -125))
+
+
+def pow2_by_division(oracle, a, M):
+    with np.errstate(under="ignore"):
+        return oracle.pow2_ceil(np.maximum(a / F(M), F(2.0 ** -126)))
+
+
+@pytest.mark.parametrize("M", [448.0, 6.0])
+def test_pow2_scale_brackets(oracle, M):
+    rng = np.random.default_rng(9 + int(M))
+    # random amaxes over the whole normal range, and amaxes within 64 ulps of
+    # M * 2**k for every k (quotients next to a power of two)
+    a1 = (F(2.0) ** rng.uniform(-110, 127, 1_000_000).astype(np.float32)).astype(np.float32)
+    k = np.arange(-120, 120, dtype=np.float64)
+    a0 = (M * 2.0 ** k).astype(np.float32)
+    d = np.arange(-64, 65, dtype=np.int64)
+    a2 = (a0.view(np.uint32).astype(np.int64)[:, None] + d[None, :]).astype(np.uint32).view(np.float32).ravel()
+    a3 = (F(2.0) ** rng.uniform(-149, -110, 100_000).astype(np.float32)).astype(np.float32)  # tiny: floor
+    a = np.concatenate([a1, a2[np.isfinite(a2) & (a2 > 0)], a3])
+    want = pow2_by_division(oracle, a, M)
+    got, decided = pow2_by_bracket(oracle, a, M)
+    bad = decided & (got != want)
+    assert not bad.any(), f"{bad.sum()} power-of-two scales differ; first a={a[bad][0]!r}"
+    assert decided[: a1.size].mean() > 0.999
+    assert not decided.all()  # the quotients next to a power of two do reach the division
+
+
+# ---- resolving a straddled bracket without the division ---------------------
+#
+# When the two brackets of an element give different e2m1 codes, exactly one
+# rounding boundary b of e2m1 (0.25, 0.75, 1.25, 1.75, 2.5, 3.5 or 5; the
+# brackets are far narrower than the gaps between them) lies between the
+# codes, and |x| is within 2**-20 of b * d.  Then e = fma(-b, d, |x|) is
+# exact (|x| - b*d fits in a handful of bits), and with hu = half an ulp of b
+# and hd = half an ulp of the float just below b (hd = hu / 2 when b = 0.25 is
+# a power of two):
+#   RN(|x|/d) > b  iff  e > hu * d;   RN(|x|/d) < b  iff  e < -hd * d;
+#   otherwise RN(|x|/d) == b, an e2m1 tie, which rounds to the even code.
+# (b has an even significand, so RN of b + hu and of b - hd is b itself.)
+
+BOUNDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+
+
+def resolve_straddle(oracle, x, d, clo, chi):
+    """Codes for elements whose bracket codes differ, by the exact fma test."""
+    k = np.minimum(clo & 7, chi & 7).astype(np.int64)   # the lower magnitude code
+    b = BOUNDS[k]
+    eb = np.floor(np.log2(b.astype(np.float64))).astype(np.int64)
+    hu = np.ldexp(np.float32(1.0), eb - 24).astype(np.float32)
+    hd = np.where(b == np.float32(0.25), hu / np.float32(2), hu).astype(np.float32)
+    ax = np.abs(x).astype(np.float64)
+    e = ax - b.astype(np.float64) * d.astype(np.float64)   # the exact fma value
+    assert np.all(np.float32(e) == e), "fma(-b, d, |x|) must be exact here"
+    up = e > (hu.astype(np.float64) * d.astype(np.float64))
+    down = e < -(hd.astype(np.float64) * d.astype(np.float64))
+    mag = np.where(up, k + 1, np.where(down, k, np.where(k % 2 == 0, k, k + 1)))
+    return (mag | (np.signbit(x).astype(np.int64) << 3)).astype(np.int32)
+
+
+@pytest.mark.parametrize("m", E2M1_MIDPOINTS)
+def test_straddle_resolution(oracle, m):
+    """Every straddled bracket of the scaled-reciprocal shortcut near each
+    e2m1 boundary, over every e4m3 scale and random g, resolved by the fma
+    test, equals the code of the plain division."""
+    rng = np.random.default_rng(int(m * 32) + 5)
+    sv = e4m3_values(oracle)
+    g = (F(2.0) ** rng.uniform(-30, 30, 48).astype(np.float32) * rng.uniform(1, 2, 48).astype(np.float32))
+    ss = np.repeat(sv, g.size)
+    gg = np.tile(g.astype(np.float32), sv.size)
+    d = (ss * gg).astype(np.float32)
+    x0 = (F(m) * d).astype(np.float32)
+    k = np.arange(-12, 13, dtype=np.int64)
+    x = (x0.view(np.uint32).astype(np.int64)[:, None] + k[None, :]).astype(np.uint32).view(np.float32).ravel()
+    ss, gg, d = np.repeat(ss, k.size), np.repeat(gg, k.size), np.repeat(d, k.size)
+    x = np.concatenate([x, -x])
+    ss, gg, d = np.concatenate([ss, ss]), np.concatenate([gg, gg]), np.concatenate([d, d])
+    with np.errstate(over="ignore", under="ignore", divide="ignore", invalid="ignore"):
+        r = (F(1) / ss) * (F(1) / gg)
+        lo, hi = x * (r * LO21), x * (r * HI21)
+    clo, chi = oracle.e2m1_round(lo), oracle.e2m1_round(hi)
+    ok = (r >= F(2.0 ** -125)) & (r <= F(2.0 ** 125)) & (clo != chi)
+    assert ok.sum() > 1000  # plenty of straddles are exercised
+    want = element_codes_by_division(oracle, x[ok], d[ok])
+    got = resolve_straddle(oracle, x[ok], d[ok], clo[ok], chi[ok])
+    assert np.array_equal(got, want), f"{(got != want).sum()} straddles resolved wrongly"
+    # the codes differ by exactly one magnitude step
+    assert np.all(np.abs((clo[ok] & 7).astype(np.int64) - (chi[ok] & 7).astype(np.int64)) == 1)

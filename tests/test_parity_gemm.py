@@ -172,3 +172,71 @@ def test_gemm_full_size_sampled(B, oracle, fmt, pair, monkeypatch):
         ref = oracle.grouped_mm_rows(fmt, backward, a, packed, scales, g, offs, rows)
         check_rows(got[rows], ref, a, Wmax, 2048 if backward else 7168,
                    f"full-size fmt={fmt} pair={pair} {'bwd' if backward else 'fwd'}")
+
+
+@pytest.mark.parametrize("backward", [False, True])
+def test_gemm_fused_gate_up_halves(B, oracle, backward):
+    """A fused gate/up expert weight [E, 2H, K] quantized as one NVFP4 tensor
+    whose rows carry their half's tensor scale (nvfp4 page: per-row scales let
+    fused gate/up projections carry the two tensor scales of their halves
+    exactly).  Forward applies the per-row scales in the epilogue, backward
+    folds them into the dequantized weight (they lie on its contraction)."""
+    T, K, H, E = 1200, 512, 256, 5
+    x, w, go, offs = make_problem(T, K, 2 * H, E, 21)
+    wf = f32(w)
+    wf[:, H:] *= np.float32(7.0)  # the up half 7x larger: distinct tensor scales
+    from fp8_microscaling_quantization_b200 import synth
+    w = synth.to_bf16_bits(wf)
+    packed = np.empty((E, 2 * H, K // 2), np.uint8)
+    scales = np.empty((E, 2 * H, K // 16), np.uint8)
+    g = np.empty((E, 2 * H), np.float32)
+    for e in range(E):
+        t_gate = np.float32(np.abs(f32(w[e, :H])).max()) / np.float32(2688.0)
+        t_up = np.float32(np.abs(f32(w[e, H:])).max()) / np.float32(2688.0)
+        assert t_up > 2 * t_gate
+        rs = np.concatenate([np.full(H, t_gate, np.float32), np.full(H, t_up, np.float32)])
+        packed[e], scales[e], g[e] = oracle.quantize_nvfp4(w[e], row_scale=rs)
+        # each half equals its own ModelOpt (per-tensor) quantization
+        pg, sg, tg = oracle.quantize_nvfp4_tensor(w[e, :H])
+        assert tg == t_gate and np.array_equal(pg, packed[e, :H]) and np.array_equal(sg, scales[e, :H])
+    fmt = oracle.FMT_NVFP4
+    a = go if backward else x
+    got, err = run_gemm(B, oracle, fmt, backward, a, packed, scales, g, offs)
+    assert err == 0
+    rows = np.arange(T)
+    ref = oracle.grouped_mm_rows(fmt, backward, a, packed, scales, g, offs, rows)
+    Wmax = max(np.abs(oracle.dequant_expert_f32(fmt, packed[e], scales[e], g[e])).max() for e in range(E))
+    end = int(offs[-1])
+    assert np.all(got[end:] == 0)
+    check_rows(got[:end], ref[:end], a, Wmax, 2 * H if backward else K, f"gate/up {'bwd' if backward else 'fwd'}")
+    if not backward:
+        # the up half's outputs are ~7x the gate half's: the scales were applied per half
+        ratio = np.abs(got[:end, H:]).mean() / np.abs(got[:end, :H]).mean()
+        assert 5.0 < ratio < 9.0
+
+
+@pytest.mark.parametrize("pair", ["0", "1"])
+def test_gemm_wait_limit_runs_out_then_recovers(B, oracle, pair, monkeypatch):
+    """Every pipeline wait of the GEMM is bounded.  With the limit cut to 1 ns
+    (BSQ_GMM_WAIT_NS) the waits run out: the kernel must record
+    BSQ_DEVERR_TIMEOUT in the error word and return, and the next call on the
+    same stream, with the normal limit, must be correct."""
+    import time
+    monkeypatch.setenv("BSQ_GMM_CTA_PAIR", pair)
+    T, K, N, E = 1024, 512, 256, 4
+    x, w, go, offs = make_problem(T, K, N, E, 23)
+    fmt = oracle.FMT_MXFP4
+    packed, scales, g = quantize_weights(oracle, fmt, w)
+    monkeypatch.setenv("BSQ_GMM_WAIT_NS", "1")
+    t0 = time.monotonic()
+    _, err = run_gemm(B, oracle, fmt, False, x, packed, scales, g, offs)
+    assert time.monotonic() - t0 < 60.0
+    assert err & 2, f"no timeout reported (err={err})"
+    monkeypatch.delenv("BSQ_GMM_WAIT_NS")
+    for backward, a in ((False, x), (True, go)):
+        got, err = run_gemm(B, oracle, fmt, backward, a, packed, scales, g, offs)
+        assert err == 0
+        ref = oracle.grouped_mm_rows(fmt, backward, a, packed, scales, g, offs, np.arange(T))
+        Wmax = max(np.abs(oracle.dequant_expert_f32(fmt, packed[e], scales[e])).max() for e in range(E))
+        end = int(offs[-1])
+        check_rows(got[:end], ref[:end], a, Wmax, N if backward else K, "after a timed-out call")

@@ -36,10 +36,13 @@ def edge_bf16_values():
 
 # ---------------------------------------------------------------- NVFP4 -----
 
-# K > 65536 takes the two-kernel form (row amax pass, then the flat quantize
-# reading the computed row scales); the rest run the one-CTA-per-row kernel.
-@pytest.mark.parametrize("rows,K", [(256, 2048), (37, 272), (5, 16), (129, 4096), (3, 40000), (1, 32768),
-                                    (1, 65536), (3, 65552), (2, 131072)])
+# Rows of up to 2048 blocks (bf16 K <= 32768) are staged whole in shared
+# memory by bulk copies (at most 4 blocks per thread: K = 8240 gives 515
+# blocks on 288 threads); longer rows up to K = 65536 run the one-CTA-per-row
+# kernel that re-reads the row from L2; K > 65536 takes the two-kernel form
+# (row amax pass, then the flat quantize reading the computed row scales).
+@pytest.mark.parametrize("rows,K", [(256, 2048), (37, 272), (5, 16), (129, 4096), (7, 8240), (3, 40000),
+                                    (1, 32768), (1, 65536), (3, 65552), (2, 131072)])
 def test_nvfp4_rowamax_bf16(B, S, oracle, rows, K):
     x = S.nvfp4_matrix(rows=rows, cols=K, seed=1000 + rows + K)
     p, s, g = B.bsq_quantize_nvfp4(dev_bf16(x))
@@ -54,7 +57,9 @@ def test_nvfp4_rowamax_bf16(B, S, oracle, rows, K):
     assert_bits_equal(host_bits(y32), oracle.dequantize_nvfp4(op, os_, og, out_dtype=oracle.F32), "dequant fp32")
 
 
-@pytest.mark.parametrize("rows,K", [(64, 1024), (3, 65552)])
+# fp32 rows are staged up to 100 KiB (K = 25600, two stages of 100 KiB);
+# K = 25616 and longer rows take the other kernels
+@pytest.mark.parametrize("rows,K", [(64, 1024), (5, 25600), (4, 25616), (3, 65552)])
 def test_nvfp4_rowamax_fp32_input(B, S, oracle, rows, K):
     rng = np.random.default_rng(5 + K)
     x = (rng.standard_normal((rows, K)) * np.exp(rng.uniform(-20, 20, (rows, 1)))).astype(np.float32)
@@ -64,6 +69,40 @@ def test_nvfp4_rowamax_fp32_input(B, S, oracle, rows, K):
     assert_bits_equal(host_bits(g), og, "row scale")
     assert_bits_equal(host_bits(s), os_, "scales")
     assert_bits_equal(host_bits(p), op, "packed")
+
+
+@pytest.mark.parametrize("fp32", [False, True])
+def test_nvfp4_boundary_hits(B, oracle, fp32):
+    """Rows whose blocks each hold 1.0 and 1/8 of it: with g = amax / 2688 the
+    block scale is 448 and the quotient of 1/8 lands on the e2m1 midpoint 0.75
+    up to the roundings of g and d, so the division-free brackets disagree in
+    every block (1024 per row, more than the kernel's redo queue holds) and the
+    plain rule decides.  Per-row, per-tensor and given (data-derived) scales."""
+    rng = np.random.default_rng(31)
+    rows, K = 6, 16384
+    x = np.zeros((rows, K), np.uint16)
+    x[:, 0::16] = 0x3F80                                   # 1.0
+    x[:, 1::16] = 0x3E00                                   # 0.125
+    x[:, 2::16] = rng.choice([0x3EC0, 0x3F40, 0x3D00], (rows, K // 16))  # 0.375, 0.75, 1/32
+    x[:, 3::16] = rng.integers(0, 0x3F80, (rows, K // 16)).astype(np.uint16)
+    x[1] = x[0] ^ 0x8000                                   # negative copy
+    x[3, 0] = 0x4000                                       # row max 2.0: quotients of 1/16 ...
+    xin = dev(f32_of(x)) if fp32 else dev_bf16(x)
+    xo = f32_of(x) if fp32 else x
+    p, s, g = B.bsq_quantize_nvfp4(xin)
+    op, os_, og = oracle.quantize_nvfp4(xo)
+    assert_bits_equal(host_bits(g), og, "row scale (hits)")
+    assert_bits_equal(host_bits(s), os_, "scales (hits)")
+    assert_bits_equal(host_bits(p), op, "packed (hits)")
+    p, s, t = B.bsq_quantize_nvfp4_tensor(xin)
+    op, os_, ot = oracle.quantize_nvfp4_tensor(xo)
+    assert_bits_equal(host_bits(t)[:1], np.array([ot], np.float32), "tensor scale (hits)")
+    assert_bits_equal(host_bits(s), os_, "tensor scales (hits)")
+    assert_bits_equal(host_bits(p), op, "tensor packed (hits)")
+    p, s, g = B.bsq_quantize_nvfp4(xin, row_scale_in=dev(og))
+    op, os_, _ = oracle.quantize_nvfp4(xo, row_scale=og)
+    assert_bits_equal(host_bits(s), os_, "given scales (hits)")
+    assert_bits_equal(host_bits(p), op, "given packed (hits)")
 
 
 def test_nvfp4_edge_values(B, oracle):
@@ -106,16 +145,24 @@ def test_nvfp4_edge_values(B, oracle):
     assert_bits_equal(host_bits(y), oracle.dequantize_nvfp4(op, os_, og, out_dtype=oracle.F32), "dequant (edges)")
 
 
-def test_nvfp4_given_row_scales(B, S, oracle):
-    x = S.linear_weight(out=96, inp=2048, seed=77)
+@pytest.mark.parametrize("rows,K", [(96, 2048), (9, 8240), (3, 40000)])
+def test_nvfp4_given_row_scales(B, S, oracle, rows, K):
+    x = S.linear_weight(out=rows, inp=K, seed=77 + K)
     rng = np.random.default_rng(8)
-    g_in = rng.uniform(1e-6, 1e-4, 96).astype(np.float32)
-    g_in[5] = 0.0
+    g_in = rng.uniform(1e-6, 1e-4, rows).astype(np.float32)
+    g_in[min(5, rows - 1)] = 0.0
+    g_in[0] = 1e-9  # block scales saturate at 448: codes of quotients far above 6
     p, s, g = B.bsq_quantize_nvfp4(dev_bf16(x), row_scale_in=dev(g_in))
     op, os_, og = oracle.quantize_nvfp4(x, row_scale=g_in)
     assert_bits_equal(host_bits(g), og, "row scale copy")
     assert_bits_equal(host_bits(s), os_, "scales")
     assert_bits_equal(host_bits(p), op, "packed")
+    # fp32 input with the same scales
+    xf = f32_of(x)
+    p, s, g = B.bsq_quantize_nvfp4(dev(xf), row_scale_in=dev(g_in))
+    op, os_, og = oracle.quantize_nvfp4(xf, row_scale=g_in)
+    assert_bits_equal(host_bits(s), os_, "scales fp32")
+    assert_bits_equal(host_bits(p), op, "packed fp32")
 
 
 def test_nvfp4_dequant_all_scale_codes(B, oracle):
@@ -130,8 +177,9 @@ def test_nvfp4_dequant_all_scale_codes(B, oracle):
         assert_bits_equal(host_bits(y), oracle.dequantize_nvfp4(packed, scales, g, out_dtype=odt), f"dequant {dt}")
 
 
-def test_nvfp4_modelopt_tensor_scale(B, S, oracle):
-    x = S.linear_weight(out=300, inp=4096, seed=78)
+@pytest.mark.parametrize("rows,K", [(300, 4096), (5, 40000)])
+def test_nvfp4_modelopt_tensor_scale(B, S, oracle, rows, K):
+    x = S.linear_weight(out=rows, inp=K, seed=78 + K)
     p, s, t = B.bsq_quantize_nvfp4_tensor(dev_bf16(x))
     op, os_, ot = oracle.quantize_nvfp4_tensor(x)
     assert_bits_equal(host_bits(t)[:1], np.array([ot], np.float32), "tensor scale")
