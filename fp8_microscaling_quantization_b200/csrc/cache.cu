@@ -14,8 +14,18 @@
 namespace bsq {
 
 // ------------------------------------------------------- quantize_cache ----
+// Per-CTA tables of the NVFP4 path (unused by the other formats).
+struct NvTables {
+    float inv[128];
+    NvBound bounds[8];
+};
+__device__ __forceinline__ void fill_nv_tables(NvTables* t) {
+    fill_inv_e4m3(t->inv);
+    fill_nv_bounds(t->bounds);
+}
+
 template <int FMT, int L>
-__device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg, float out[8]);
+__device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg, const NvTables* tab, float out[8]);
 
 // S lanes per row (S a power of two, 2 <= S <= 32; 32/S rows per warp); lane
 // i of a row walks the chunks i, i + S, ...  of the zero-padded row, so the
@@ -26,6 +36,11 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
                                                          int64_t C) {
     constexpr int L = BLOCK / 8;
     constexpr int RPW = 32 / S;  // rows per warp
+    __shared__ NvTables tab;
+    if (FMT == BSQ_NVFP4) {
+        fill_nv_tables(&tab);
+        __syncthreads();
+    }
     const int lane = threadIdx.x & 31;
     const int sl = lane % S;
     const int64_t nb = (C + BLOCK - 1) / BLOCK;
@@ -50,7 +65,7 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
                     m = fmaxf(m, amax8(v));
                 }
             }
-            m = group_max<S>(m);
+            m = (S == 32) ? warp_max_nonneg(m) : group_max<S>(m);
             g = __fdiv_rn(m, kNvGlobalDiv);
             rg = nv_recip_or_zero(g);
         }
@@ -66,7 +81,7 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
                 for (int j = 0; j < 8; ++j) v[j] = 0.0f;
             }
             float out[8];
-            cache_chunk<FMT, L>(v, g, rg, out);
+            cache_chunk<FMT, L>(v, g, rg, &tab, out);
             if (row_ok && c < cpr && n > 0) {
                 if (VEC && n >= 8) store8(yr + c * 8, out);
                 else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
@@ -76,12 +91,16 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
 }
 
 // Fake-quant of one 8-element chunk in registers (the block's lanes are
-// adjacent; g is the row scale for NVFP4).
+// adjacent; g is the row scale for NVFP4, rg = nv_recip_or_zero(g)).  The
+// power-of-two scales and the NVFP4 codes are taken without a division (see
+// pow2_scale_fast and nv_block_codes_fast); the dequantized value is one
+// multiply by the positive scale, folded with +0.0 into an fma so that code 8
+// (-0.0 from the hardware decode) gives the table's +0.0.
 template <int FMT, int L>
-__device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg, float out[8]) {
+__device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg, const NvTables* tab, float out[8]) {
     const float amax_b = group_max<L>(amax8(v));
     if (FMT == BSQ_FP8) {
-        const float p = pow2_scale(amax_b, kE4M3Max);
+        const float p = pow2_scale_fast(amax_b, kE4M3Max, 1.0f / kE4M3Max);
         const float inv = exp2_int(127 - f32_biased_exp(p));
 #pragma unroll
         for (int j = 0; j < 8; j += 2) {
@@ -90,27 +109,45 @@ __device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg,
             out[j + 1] = d.y * p;
         }
     } else if (FMT == BSQ_MXFP4) {
-        const float p = pow2_scale(amax_b, kE2M1Max);
+        const float p = pow2_scale_fast(amax_b, kE2M1Max, 1.0f / kE2M1Max);
         const float inv = exp2_int(127 - f32_biased_exp(p));
         float q[8], e[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) q[j] = v[j] * inv;
-        e2m1x8_decode_hw(e2m1x8_encode_hw(q), e);
-        // e * p is exact
+        e2m1x8_decode_raw(e2m1x8_encode_hw(q), e);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(e[j], p);
+        for (int j = 0; j < 8; ++j) out[j] = __fmaf_rn(e[j], p, 0.0f);  // exact product
     } else {
         if (g == 0.0f) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) out[j] = 0.0f;
         } else {
-            const float s = e4m3_decode(nv_scale_code(amax_b, g, rg));
-            const float d = __fmul_rn(s, g);
-            float e[8];
-            e2m1x8_decode_hw(e2m1x8_of_quotient(v, d), e);
-            // (e2m1 * s) is exact (and +0 for code 8), then one rounding by g
+            const uint32_t sc = nv_scale_code(amax_b, g, rg);
+            const float s = e4m3x2_decode_hw(sc).x;
+            uint32_t codes;
+            const float r = __fmul_rn(tab->inv[sc], rg);
+            if (r >= 2.3509887e-38f && r <= 4.2535296e37f) {
+                const float2 rlo = make_float2(__fmul_rn(r, 0.99999952f), __fmul_rn(r, 0.99999952f));
+                const float2 rhi = make_float2(__fmul_rn(r, 1.00000048f), __fmul_rn(r, 1.00000048f));
+                float lo[8], hi[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(__fmul_rn(e[j], s), g);
+                for (int j = 0; j < 8; j += 2) {
+                    const float2 a = mul_f32x2(make_float2(v[j], v[j + 1]), rlo);
+                    const float2 b = mul_f32x2(make_float2(v[j], v[j + 1]), rhi);
+                    lo[j] = a.x; lo[j + 1] = a.y;
+                    hi[j] = b.x; hi[j + 1] = b.y;
+                }
+                codes = e2m1x8_encode_hw(lo);
+                const uint32_t diff = codes ^ e2m1x8_encode_hw(hi);
+                if (diff) codes = nv_settle_straddles_regs(codes, diff, v, __fmul_rn(s, g), tab->bounds);
+            } else {
+                codes = e2m1x8_of_quotient(v, __fmul_rn(s, g));
+            }
+            float e[8];
+            e2m1x8_decode_raw(codes, e);
+            // (e2m1 * s) is exact, then one rounding by g (+0.0 for code 8)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) out[j] = __fmaf_rn(__fmul_rn(e[j], s), g, 0.0f);
         }
     }
 }
@@ -140,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 8) cache_flat_kernel(const T* __rest
             const int64_t c = base + u * stride + lane;
             float v[8], out[8];
             raw[u].get(v);
-            cache_chunk<FMT, L>(v, 0.0f, 0.0f, out);
+            cache_chunk<FMT, L>(v, 0.0f, 0.0f, nullptr, out);
             if (c < nchunks) store8(y + c * 8, out);
         }
     }
@@ -154,6 +191,11 @@ __global__ void __launch_bounds__(kThreads) cache_row_kernel(const T* __restrict
                                                              int64_t rows, int64_t C) {
     constexpr int L = BLOCK / 8;
     constexpr int RPW = 32 / S;
+    __shared__ NvTables tab;
+    if (FMT == BSQ_NVFP4) {
+        fill_nv_tables(&tab);
+        __syncthreads();
+    }
     const int lane = threadIdx.x & 31;
     const int sl = lane % S;
     const int64_t cpr = ((C + BLOCK - 1) / BLOCK) * L;
@@ -181,7 +223,7 @@ __global__ void __launch_bounds__(kThreads) cache_row_kernel(const T* __restrict
         }
         float g = 0.0f, rg = 0.0f;
         if (FMT == BSQ_NVFP4) {
-            g = __fdiv_rn(group_max<S>(m), kNvGlobalDiv);
+            g = __fdiv_rn(S == 32 ? warp_max_nonneg(m) : group_max<S>(m), kNvGlobalDiv);
             rg = nv_recip_or_zero(g);
         }
 #pragma unroll
@@ -190,7 +232,7 @@ __global__ void __launch_bounds__(kThreads) cache_row_kernel(const T* __restrict
             const int64_t c = sl + (int64_t)i * S;
             const int64_t n = C - c * 8;
             float out[8];
-            cache_chunk<FMT, L>(v[i], g, rg, out);
+            cache_chunk<FMT, L>(v[i], g, rg, &tab, out);
             if (row_ok && c < cpr && n > 0) {
                 if (VEC && n >= 8) store8(yr + c * 8, out);
                 else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);

@@ -86,6 +86,13 @@ __device__ __forceinline__ float group_max(float m) {
     return m;
 }
 
+// Max over the 32 lanes of a warp of a non-negative binary32 (an amax): the
+// bit patterns of non-negative floats order as unsigned integers, so one
+// redux.sync does it.
+__device__ __forceinline__ float warp_max_nonneg(float m) {
+    return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(m)));
+}
+
 __device__ __forceinline__ float block_reduce_max(float m, float* smem /* >= 32 floats */) {
     m = group_max<32>(m);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -116,6 +123,21 @@ __device__ __forceinline__ float pow2_scale(float amax_b, float fmt_max) {
     float a = __fdiv_rn(amax_b, fmt_max);
     if (a < kF32MinNormal) a = kF32MinNormal;
     return pow2_ceil_normal(a);
+}
+
+// The same without the division: q = RN(a * inv_max) (inv_max = RN(1 /
+// fmt_max)) is within two roundings of a / fmt_max and RN(a / fmt_max) within
+// one, and pow2ceil is monotone, so when the brackets RN(q * (1 -+ 2**-21))
+// have the same power-of-two ceiling, that is the rule's value.  Otherwise (a
+// quotient next to a power of two) or for q < 2**-125, the division.
+__device__ __forceinline__ float pow2_scale_fast(float amax_b, float fmt_max, float inv_max) {
+    const float q = __fmul_rn(amax_b, inv_max);
+    if (q >= 2.3509887e-38f /* 2**-125 */) {
+        const float plo = pow2_ceil_normal(__fmul_rn(q, 0.99999952f));
+        const float phi = pow2_ceil_normal(__fmul_rn(q, 1.00000048f));
+        if (plo == phi) return plo;
+    }
+    return pow2_scale(amax_b, fmt_max);
 }
 
 // NVFP4 block scale byte: e4m3(max((amax_b / 6) / g, 2**-9)).
@@ -367,6 +389,30 @@ __device__ __forceinline__ void fill_nv_bounds(NvBound* t) {
         t[k].hd = (k == 0) ? exp2_int(eb - 25) : exp2_int(eb - 24);
         t[k].pad = 0.0f;
     }
+}
+
+// Element i (0..7, not known at compile time) of 8 values in registers.
+__device__ __forceinline__ float pick8(const float v[8], int i) {
+    float x = v[0];
+#pragma unroll
+    for (int j = 1; j < 8; ++j) x = (i == j) ? v[j] : x;
+    return x;
+}
+
+// nv_settle_straddles for 8 elements held in registers (v).
+__device__ __forceinline__ uint32_t nv_settle_straddles_regs(uint32_t clo, uint32_t diff, const float v[8], float d,
+                                                             const NvBound* bounds) {
+    while (diff) {
+        const int sh = (__ffs(diff) - 1) & ~3;
+        diff &= ~(0xFu << sh);
+        const uint32_t cl = (clo >> sh) & 0xFu;
+        const uint32_t k = cl & 7u;
+        const NvBound bd = bounds[k];
+        const float e = __fmaf_rn(-bd.b, d, fabsf(pick8(v, sh >> 2)));
+        const uint32_t mag = (e > __fmul_rn(bd.hu, d)) ? k + 1u : ((e < -__fmul_rn(bd.hd, d)) ? k : ((k + 1u) & ~1u));
+        clo = (clo & ~(0xFu << sh)) | (((cl & 8u) | mag) << sh);
+    }
+    return clo;
 }
 
 template <typename T>

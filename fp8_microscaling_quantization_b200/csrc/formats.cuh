@@ -136,6 +136,23 @@ __device__ __forceinline__ void e2m1x8_decode_hw(uint32_t w, float v[8]) {
 }
 
 
+// The same decode without the +0.0: code 8 gives -0.0 (for callers that fold
+// the sign of zero into a later fma with +0.0).
+__device__ __forceinline__ void e2m1x8_decode_raw(uint32_t w, float v[8]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t h2;
+        asm("{\n\t.reg .b8 t;\n\t"
+            "cvt.u8.u32 t, %1;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+            : "=r"(h2)
+            : "r"(w >> (8 * i)));
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
 // e8m0 byte -> 2**(code - 127) as binary32 (code 0 is the subnormal 2**-127,
 // 0xFF is NaN).
 __device__ __forceinline__ float e8m0_decode(uint32_t c) {

@@ -195,13 +195,12 @@ __global__ void __launch_bounds__(NT, MINB)
     if (MODE == 1) {
         float m = 0.0f;
         for (int i = tid; i < npartial; i += nt) m = fmaxf(m, partial[i]);
-        m = group_max<32>(m);
+        m = warp_max_nonneg(m);
         if (lane == 0) red[0][warp] = m;
     }
     __syncthreads();
     if (MODE == 1) {
-        float m = lane < nw ? red[0][lane] : 0.0f;
-        m = group_max<32>(m);
+        const float m = warp_max_nonneg(lane < nw ? red[0][lane] : 0.0f);
         g_t = __fdiv_rn(m, kNvGlobalDiv);
         rg_t = nv_recip_or_zero(g_t);
         if (blockIdx.x == 0 && tid == 0) g_out[0] = g_t;
@@ -252,11 +251,10 @@ __global__ void __launch_bounds__(NT, MINB)
         }
         float g;
         if (MODE == 2) {
-            m = group_max<32>(m);
+            m = warp_max_nonneg(m);
             if (lane == 0) red[i & 1][warp] = m;
             __syncthreads();
-            float mm = lane < nw ? red[i & 1][lane] : 0.0f;
-            mm = group_max<32>(mm);
+            const float mm = warp_max_nonneg(lane < nw ? red[i & 1][lane] : 0.0f);
             g = __fdiv_rn(mm, kNvGlobalDiv);
         } else if (MODE == 0) {
             g = g_in[r];
@@ -319,9 +317,12 @@ static StagedPlan staged_plan(int64_t K) {
     const int64_t row_bytes = K * (int64_t)sizeof(T);
     if (bpr < 1 || bpr > (int64_t)kStgMaxThreads * kStgMaxBpt || row_bytes > 100 * 1024) return p;
     const int64_t stage_bytes = (row_bytes + 127) / 128 * 128;
-    const int bpt = (int)((bpr + kStgMaxThreads - 1) / kStgMaxThreads);
+    // as many blocks per thread as allowed (the per-row work of a thread is
+    // shared by more blocks), but at least 64 threads
+    const int bpt = (int)std::max<int64_t>(1, std::min<int64_t>(kStgMaxBpt, bpr / 64));
     const int64_t per = (bpr + bpt - 1) / bpt;
     p.nt = (int)((per + 31) / 32 * 32);
+    if (p.nt > kStgMaxThreads) return StagedPlan();
     // per CTA: the stages, under 1 KiB of static shared memory and 1 KiB the
     // hardware reserves, against the 228 KiB of an SM
     if (p.nt <= 384 && 3 * (2 * stage_bytes + 4 * 1024) <= 228 * 1024) {
