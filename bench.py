@@ -785,10 +785,18 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
         y = torch.empty_like(x)
         n = x.numel()
         nb = 2 * n + n // 2 + n // 16 + 4 * 256
-        out["nvfp4_256x2048"] = {
-            "quantize": rec(timed(lambda: bsq.bsq_quantize_nvfp4(x, packed=p, scales=s, row_scale_out=r), 50, True), nb),
-            "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_nvfp4(p, s, r, y=y), 50, True), nb),
-            "note": "latency-bound (1.3 MB); L2 flushed before every launch"}
+        q_ms = timed(lambda: bsq.bsq_quantize_nvfp4(x, packed=p, scales=s, row_scale_out=r), 50, True)
+        d_ms = timed(lambda: bsq.bsq_dequantize_nvfp4(p, s, r, y=y), 50, True)
+        # the latency floor at this size: a device-to-device copy of the
+        # input, timed the same way (the quantize reads it and writes a
+        # quarter of it; the dequantize the reverse)
+        c_ms = timed(lambda: y.copy_(x), 50, True)
+        qr, dr = rec(q_ms, nb), rec(d_ms, nb)
+        for rr, ms in ((qr, q_ms), (dr, d_ms)):
+            rr["same_size_copy_us"] = round(c_ms * 1e3, 2)
+            rr["frac_of_copy"] = round(c_ms / ms, 4)
+        out["nvfp4_256x2048"] = {"quantize": qr, "dequantize_bf16": dr,
+                                 "note": "latency-bound (1.3 MB); L2 flushed before every launch"}
 
     if want("mxfp8"):
         g = torch.Generator(device=dev)

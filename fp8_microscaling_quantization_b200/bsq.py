@@ -18,10 +18,12 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-lib_path = os.path.join(_HERE, "libbsq.so")
+# BSQ_LIBRARY may name another build of the same library, e.g. the
+# bounds-checking libbsq_debug.so
+lib_path = os.environ.get("BSQ_LIBRARY") or os.path.join(_HERE, "libbsq.so")
 
 if not os.path.exists(lib_path):
-    raise ImportError(f"libbsq.so is not built at {lib_path}; run "
+    raise ImportError(f"libbsq is not built at {lib_path}; run "
                       "`python -m fp8_microscaling_quantization_b200.build` (nvcc, sm_100a)")
 
 _L = ctypes.CDLL(lib_path)
@@ -59,6 +61,7 @@ _SIGS = {
     "bsq_status_string": (ctypes.c_char_p, [_I32]),
     "bsq_last_error": (ctypes.c_char_p, []),
     "bsq_version": (_I32, []),
+    "bsq_debug_counters": (_I32, [_P, _P]),
     "bsq_quantize_nvfp4": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _P, _P]),
     "bsq_nvfp4_tensor_scratch_bytes": (_SZ, [_I64, _I64]),
     "bsq_quantize_nvfp4_tensor": (_I32, [_P, _I32, _I64, _I64, _P, _P, _P, _P, _SZ, _P]),
@@ -98,6 +101,14 @@ def bsq_last_error() -> str:
 
 def bsq_version() -> int:
     return _L.bsq_version()
+
+
+def bsq_debug_counters():
+    """(failed index checks, code of the first) since the last call, in a
+    BSQ_DEBUG build; raises BsqError (unsupported) in a normal build."""
+    c, f = ctypes.c_uint32(0), ctypes.c_uint32(0)
+    _call("bsq_debug_counters", ctypes.byref(c), ctypes.byref(f))
+    return int(c.value), int(f.value)
 
 
 def _call(name, *args):

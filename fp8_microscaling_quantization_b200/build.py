@@ -1,6 +1,6 @@
 """Build libbsq.so in-tree with nvcc for sm_100a.
 
-    python -m fp8_microscaling_quantization_b200.build [--force]
+    python -m fp8_microscaling_quantization_b200.build [--force] [--debug]
 
 Flags: -gencode arch=compute_100a,code=sm_100a, -O3, -lineinfo, no fast-math
 (IEEE division, denormals kept), -fmad=false (no multiply-add contraction, so
@@ -18,8 +18,11 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libbsq.so")
+# the bounds-checking build (-DBSQ_DEBUG): every checked index is tested
+# against its extent, a failure is counted, not trapped (csrc/debug.cuh)
+LIB_DEBUG = os.path.join(HERE, "libbsq_debug.so")
 SOURCES = ["abi.cu", "flat.cu", "nvfp4.cu", "static.cu", "kv_cache.cu", "cache.cu", "grouped_mm.cu"]
-HEADERS = ["common.cuh", "formats.cuh", "host_util.h", "tcgen05.cuh"]
+HEADERS = ["common.cuh", "formats.cuh", "host_util.h", "tcgen05.cuh", "debug.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -42,10 +45,10 @@ def _inputs():
     return files
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
@@ -55,13 +58,18 @@ def _wait_all(procs):
         raise subprocess.CalledProcessError(1, failed[0])
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
-    """Compile every source (in parallel, one nvcc per file) and link."""
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, extra_flags=None, debug: bool = False) -> str:
+    """Compile every source (in parallel, one nvcc per file) and link;
+    debug=True builds the bounds-checking libbsq_debug.so instead."""
+    lib = LIB_DEBUG if debug else LIB
+    if debug:
+        extra_flags = list(extra_flags or []) + ["-DBSQ_DEBUG"]
+    if not force and up_to_date(lib):
+        return lib
     objs, cmds = [], []
+    tag = "dbg." if debug else ""
     for src in SOURCES:
-        obj = os.path.join(CSRC, src.replace(".cu", f".{os.getpid()}.o"))
+        obj = os.path.join(CSRC, src.replace(".cu", f".{tag}{os.getpid()}.o"))
         cmds.append([nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", os.path.join(ROOT, "include"), "-c",
                      os.path.join(CSRC, src), "-o", obj])
         objs.append(obj)
@@ -75,16 +83,16 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
             _wait_all(running[:1])
             running = running[1:]
     _wait_all(running)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler", "-fPIC", *objs, "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
     for o in objs:
         os.remove(o)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
+    build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv)

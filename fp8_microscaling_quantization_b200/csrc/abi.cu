@@ -56,3 +56,32 @@ BSQ_API const char* bsq_last_error(void) { return g_last_error; }
 
 BSQ_API int bsq_version(void) { return 1; }
 
+#ifdef BSQ_DEBUG
+// each unit's collector (debug builds only), defined next to its kernels
+cudaError_t bsq_dbg_take_flat(uint32_t*, uint32_t*);
+cudaError_t bsq_dbg_take_nvfp4(uint32_t*, uint32_t*);
+cudaError_t bsq_dbg_take_static(uint32_t*, uint32_t*);
+cudaError_t bsq_dbg_take_kv(uint32_t*, uint32_t*);
+cudaError_t bsq_dbg_take_cache(uint32_t*, uint32_t*);
+cudaError_t bsq_dbg_take_gmm(uint32_t*, uint32_t*);
+
+BSQ_API bsq_status bsq_debug_counters(uint32_t* count, uint32_t* first_code) {
+    if (!count || !first_code) return fail(BSQ_ERR_INVALID_ARG, "bsq_debug_counters: null pointer");
+    *count = 0;
+    *first_code = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    cudaError_t (*take[])(uint32_t*, uint32_t*) = {bsq_dbg_take_flat, bsq_dbg_take_nvfp4, bsq_dbg_take_static,
+                                                  bsq_dbg_take_kv, bsq_dbg_take_cache, bsq_dbg_take_gmm};
+    for (auto f : take)
+        if (e == cudaSuccess) e = f(count, first_code);
+    if (e != cudaSuccess) return fail(BSQ_ERR_CUDA, "bsq_debug_counters: %s", cudaGetErrorString(e));
+    return BSQ_OK;
+}
+#else
+BSQ_API bsq_status bsq_debug_counters(uint32_t* count, uint32_t* first_code) {
+    if (count) *count = 0;
+    if (first_code) *first_code = 0;
+    return fail(BSQ_ERR_UNSUPPORTED, "bsq_debug_counters: not a BSQ_DEBUG build");
+}
+#endif
+

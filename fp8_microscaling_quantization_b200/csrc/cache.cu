@@ -8,6 +8,8 @@
 #include <cstring>
 #include <mutex>
 
+#define BSQ_DBG_FILE 5
+#include "debug.cuh"
 #include "common.cuh"
 #include "tcgen05.cuh"
 
@@ -83,8 +85,10 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
             float out[8];
             cache_chunk<FMT, L>(v, g, rg, &tab, out);
             if (row_ok && c < cpr && n > 0) {
-                if (VEC && n >= 8) store8(yr + c * 8, out);
-                else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
+                if (BSQ_DOK(r < rows && c * 8 < C)) {
+                    if (VEC && n >= 8) store8(yr + c * 8, out);
+                    else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
+                }
             }
         }
     }
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 8) cache_flat_kernel(const T* __rest
             float v[8], out[8];
             raw[u].get(v);
             cache_chunk<FMT, L>(v, 0.0f, 0.0f, nullptr, out);
-            if (c < nchunks) store8(y + c * 8, out);
+            if (c < nchunks && BSQ_DOK(c * 8 + 8 <= nchunks * 8)) store8(y + c * 8, out);
         }
     }
 }
@@ -234,8 +238,10 @@ __global__ void __launch_bounds__(kThreads) cache_row_kernel(const T* __restrict
             float out[8];
             cache_chunk<FMT, L>(v[i], g, rg, &tab, out);
             if (row_ok && c < cpr && n > 0) {
-                if (VEC && n >= 8) store8(yr + c * 8, out);
-                else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
+                if (BSQ_DOK(r < rows && c * 8 < C)) {
+                    if (VEC && n >= 8) store8(yr + c * 8, out);
+                    else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
+                }
             }
         }
     }
@@ -329,3 +335,7 @@ BSQ_API bsq_status bsq_quantize_cache_backward(const void* grad_out, void* grad_
     if (e != cudaSuccess) return fail(BSQ_ERR_CUDA, "bsq_quantize_cache_backward: %s", cudaGetErrorString(e));
     return BSQ_OK;
 }
+
+#ifdef BSQ_DEBUG
+cudaError_t bsq_dbg_take_cache(uint32_t* count, uint32_t* first) { return bsq::dbg_take(count, first); }
+#endif

@@ -15,6 +15,8 @@
 #include <cstring>
 #include <mutex>
 
+#define BSQ_DBG_FILE 1
+#include "debug.cuh"
 #include "common.cuh"
 #include "tcgen05.cuh"
 
@@ -53,7 +55,7 @@ __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restric
                 const uint32_t packed = e2m1x8_encode_hw(q);
                 if (c < nchunks) {
                     reinterpret_cast<uint32_t*>(codes)[c] = packed;
-                    if ((lane % L) == 0) scales[c / L] = (uint8_t)(e + 127);
+                    if ((lane % L) == 0 && BSQ_DOK(c / L < nchunks / L)) scales[c / L] = (uint8_t)(e + 127);
                 }
             } else if (FMT == 3) {
                 // MXFP8: values above 448 saturate (cvt ... satfinite)
@@ -66,7 +68,7 @@ __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restric
                       (e4m3x2_encode_hw(vu[6] * inv, vu[7] * inv) << 16);
                 if (c < nchunks) {
                     reinterpret_cast<uint2*>(codes)[c] = w;
-                    if ((lane % L) == 0) scales[c / L] = (uint8_t)(e + 127);
+                    if ((lane % L) == 0 && BSQ_DOK(c / L < nchunks / L)) scales[c / L] = (uint8_t)(e + 127);
                 }
             } else {
                 const float p = pow2_scale(amax_b, kE4M3Max);
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restric
                       (e4m3x2_encode_hw(vu[6] * inv, vu[7] * inv) << 16);
                 if (c < nchunks) {
                     reinterpret_cast<uint2*>(codes)[c] = w;
-                    if ((lane % L) == 0) scales[c / L] = (uint8_t)f32_biased_exp(p);
+                    if ((lane % L) == 0 && BSQ_DOK(c / L < nchunks / L)) scales[c / L] = (uint8_t)f32_biased_exp(p);
                 }
             }
         }
@@ -120,8 +122,9 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __rest
                     w1[u] = t.y;
                 }
                 const int64_t blk = (it * EPI) / BLOCK;
-                sc[u] = scales[blk];
-                if (FMT == FMT_NV) gr[u] = g[fdiv((uint32_t)blk, bpr)];
+                if (BSQ_DOK(blk * BLOCK < nitems * EPI)) sc[u] = scales[blk];
+                if (FMT == FMT_NV && BSQ_DOK((int64_t)fdiv((uint32_t)blk, bpr) * bpr.d * BLOCK < nitems * EPI))
+                    gr[u] = g[fdiv((uint32_t)blk, bpr)];
             }
         }
 #pragma unroll
@@ -149,6 +152,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __rest
                     v[j] = (FMT == FMT_MX) ? __fmul_rn(e[j], s) : __fmul_rn(__fmul_rn(e[j], s), gr[u]);
             }
             TOUT* dst = y + it * EPI;
+            if (!BSQ_DOK(it < nitems)) continue;
             if (sizeof(TOUT) == 2) {
                 store8(reinterpret_cast<uint16_t*>(dst), v);
             } else {
@@ -310,3 +314,6 @@ BSQ_API bsq_status bsq_dequantize_fp8(const uint8_t* codes_e4m3, const uint8_t* 
     return check_launch("bsq_dequantize_fp8");
 }
 
+#ifdef BSQ_DEBUG
+cudaError_t bsq_dbg_take_flat(uint32_t* count, uint32_t* first) { return bsq::dbg_take(count, first); }
+#endif

@@ -52,6 +52,8 @@
 #include <cstdlib>
 #include <mutex>
 
+#define BSQ_DBG_FILE 6
+#include "debug.cuh"
 #include "formats.cuh"
 #include "host_util.h"
 #include "tcgen05.cuh"
@@ -300,6 +302,12 @@ __device__ __forceinline__ void load_unit(Unit& u, const Args& a, const Tile& ti
         row = (int64_t)ti.e * a.N + ks * BK + r;
         kcol = ti.f0 + c;
     }
+    if (!BSQ_DOK(row < (int64_t)a.E * a.N && kcol + kUE <= a.K)) {  // debug build: skip, record
+        u.w[0] = u.w[kUE / 8 - 1] = 0u;
+        u.sc = 0u;
+        u.g = 0.0f;
+        return;
+    }
     const uint8_t* src = a.packed + row * (a.K / 2) + kcol / 2;
     if (kUE == 32) {
         const uint4 t = __ldg(reinterpret_cast<const uint4*>(src));
@@ -460,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                     float v = __uint_as_float(r[j]);
                     if (FMT == BSQ_NVFP4 && DIR == BSQ_FWD) v *= gf;
                     const __nv_bfloat16 h = __float2bfloat16_rn(v);
-                    if (j < nv) *p = *reinterpret_cast<const uint16_t*>(&h);
+                    if (j < nv && BSQ_DOK(ti.tok0 + c * 16 + j < args.T && f < out_w)) *p = *reinterpret_cast<const uint16_t*>(&h);
                     p += out_w;
                 }
             }
@@ -799,3 +807,7 @@ BSQ_API bsq_status bsq_grouped_mm_fp4(bsq_format fmt, bsq_dir dir, const void* a
     return dir == BSQ_FWD ? launch_gmm<BSQ_NVFP4, BSQ_FWD, 1>(tmap, args, max_groups, s)
                           : launch_gmm<BSQ_NVFP4, BSQ_BWD, 1>(tmap, args, max_groups, s);
 }
+
+#ifdef BSQ_DEBUG
+cudaError_t bsq_dbg_take_gmm(uint32_t* count, uint32_t* first) { return bsq::dbg_take(count, first); }
+#endif

@@ -18,6 +18,8 @@
 // while the previous unit runs, so the codes of a unit are requested without
 // first waiting for a pointer.  e2m1 codes are decoded by the hardware
 // e2m1 -> f16x2 conversion.
+#define BSQ_DBG_FILE 4
+#include "debug.cuh"
 #include "common.cuh"
 
 namespace bsq {
@@ -68,7 +70,7 @@ __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const uint8_t* con
         float na = a;
         if (nxt < nunits) {
             nb = fdiv((uint32_t)nxt, units_per_block);
-            if (nb != b) {
+            if (nb != b && BSQ_DOK((int64_t)nb * units_per_block.d < nunits)) {
                 nvb = values[nb];
                 nsb = scales[nb];
                 na = ld_f32_any(amax[nb]);
@@ -80,7 +82,7 @@ __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const uint8_t* con
         for (int u = 0; u < U; ++u) {
             const uint32_t o = o0 + u * kThreads;
             w[u] = sc[u] = 0u;
-            if (o < items_per_block) {
+            if (o < items_per_block && BSQ_DOK(((o * EPI) >> 4) < items_per_block * EPI / 16)) {
                 w[u] = ld_codes(vb, o, EPI / 2);
                 // element o * EPI of the block: scale byte (o * EPI) / 16 of
                 // the row-major [rows, 8] scales
@@ -99,6 +101,7 @@ __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const uint8_t* con
 #pragma unroll
             for (int i = 0; i < EPI; ++i) v[i] = __fmul_rn(__fmul_rn(e[i], s), g);
             TOUT* dst = yb + (int64_t)o * EPI;
+            if (!BSQ_DOK((int64_t)b * units_per_block.d < nunits && o < items_per_block)) continue;
             if (sizeof(TOUT) == 2) {
                 uint4 o4;
                 o4.x = pack_bf16x2(v[0], v[1]);
@@ -150,3 +153,7 @@ BSQ_API bsq_status bsq_dequantize_kv_cache_nvfp4(const uint8_t* const* values, c
                                                              (float*)y);
     return check_launch(fn);
 }
+
+#ifdef BSQ_DEBUG
+cudaError_t bsq_dbg_take_kv(uint32_t* count, uint32_t* first) { return bsq::dbg_take(count, first); }
+#endif

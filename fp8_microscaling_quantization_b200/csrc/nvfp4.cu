@@ -9,6 +9,8 @@
 #include <cstring>
 #include <mutex>
 
+#define BSQ_DBG_FILE 2
+#include "debug.cuh"
 #include "common.cuh"
 #include "tcgen05.cuh"
 
@@ -54,8 +56,10 @@ __global__ void __launch_bounds__(kRowThreads) nv_rowamax_quant_kernel(const T* 
             load16(xr + blk * 16, v);
             uint32_t sb;
             const uint2 pk = nv_quant_block(v, g, rg, &sb);
-            reinterpret_cast<uint2*>(packed + r * (K / 2))[blk] = pk;
-            scales[r * bpr + blk] = (uint8_t)sb;
+            if (BSQ_DOK(r < rows && blk < bpr)) {
+                reinterpret_cast<uint2*>(packed + r * (K / 2))[blk] = pk;
+                scales[r * bpr + blk] = (uint8_t)sb;
+            }
         }
     }
 }
@@ -143,11 +147,12 @@ __global__ void __launch_bounds__(kThreads) nv_flat_quant_kernel(const T* __rest
             uint32_t sb;
             const float rg = (MODE == 1) ? rg_tensor : nv_recip_or_zero(g[u]);
             const uint2 pk = nv_quant_block(v[u], g[u], rg, &sb);
+            if (!BSQ_DOK(b < nblocks)) continue;
             reinterpret_cast<uint2*>(packed)[b] = pk;
             scales[b] = (uint8_t)sb;
             if (MODE == 0) {
                 const uint32_t row = fdiv((uint32_t)b, bpr);
-                if ((uint32_t)b == row * bpr.d) g_out[row] = g[u];
+                if ((uint32_t)b == row * bpr.d && BSQ_DOK((int64_t)row * bpr.d < nblocks)) g_out[row] = g[u];
             }
         }
     }
@@ -257,18 +262,18 @@ __global__ void __launch_bounds__(NT, MINB)
             const float mm = warp_max_nonneg(lane < nw ? red[i & 1][lane] : 0.0f);
             g = __fdiv_rn(mm, kNvGlobalDiv);
         } else if (MODE == 0) {
-            g = g_in[r];
+            g = BSQ_DOK(r < rows) ? g_in[r] : 0.0f;
         } else {
             g = g_t;
         }
-        if (MODE != 1 && tid == 0) g_out[r] = g;
+        if (MODE != 1 && tid == 0 && BSQ_DOK(r < rows)) g_out[r] = g;
         const float rg = (MODE == 1) ? rg_t : nv_recip_or_zero(g);
         uint8_t* prow = packed + r * (int64_t)(K / 2);
         uint8_t* srow = scales + r * (int64_t)bpr;
         uint32_t redo_self = 0u;
 #pragma unroll
         for (int j = 0; j < kStgMaxBpt; ++j) {
-            if (j < myb) {
+            if (j < myb && BSQ_DOK(tid + j * nt < bpr && (uint32_t)(tid + j * nt + 1) * kBlkBytes <= stage_bytes)) {
                 const int b = tid + j * nt;
                 const uint32_t blk = xs + (uint32_t)b * kBlkBytes;
                 uint32_t sb = 0u;
@@ -567,4 +572,6 @@ BSQ_API bsq_status bsq_quantize_nvfp4_tensor_noalloc(const void* x, bsq_dtype xt
                                "bsq_quantize_nvfp4_tensor_noalloc");
 }
 
-
+#ifdef BSQ_DEBUG
+cudaError_t bsq_dbg_take_nvfp4(uint32_t* count, uint32_t* first) { return bsq::dbg_take(count, first); }
+#endif

@@ -19,6 +19,8 @@
 // CTA, since f is fixed per launch; the e2m1 codes of x / sq come from the
 // division-free exact quotient rounding, and decode back through the
 // hardware e2m1 -> f16x2 conversion.
+#define BSQ_DBG_FILE 3
+#include "debug.cuh"
 #include "common.cuh"
 
 namespace bsq {
@@ -51,7 +53,7 @@ __global__ void __launch_bounds__(kThreads) nv_static_fq_kernel(const T* __restr
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t c = base + u * stride;
-            if (c < nchunks) {
+            if (c < nchunks && BSQ_DOK((c >> 1) < (nchunks + 1) / 2)) {
                 load8(x + c * 8, v[u]);
                 a[u] = __ldg(block_amax + (c >> 1));
             } else {
@@ -109,3 +111,7 @@ BSQ_API bsq_status bsq_fake_quantize_nvfp4_static(const void* x, bsq_dtype t, in
                                                    (float*)y);
     return check_launch(fn);
 }
+
+#ifdef BSQ_DEBUG
+cudaError_t bsq_dbg_take_static(uint32_t* count, uint32_t* first) { return bsq::dbg_take(count, first); }
+#endif

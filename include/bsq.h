@@ -67,6 +67,17 @@ const char* bsq_status_string(bsq_status s);
 const char* bsq_last_error(void);
 int bsq_version(void);
 
+/* Index-check counters of the bounds-checking build (compiled with
+ * -DBSQ_DEBUG, shipped as libbsq_debug.so; the quantization pages have no
+ * counterpart: this is a diagnostic of the library itself).  In that build
+ * every checked device access first tests its index against the extent the
+ * kernel was given; a failing check skips the access (no trap) and is
+ * counted.  Synchronises the current device, stores the number of failed
+ * checks since the previous call in *count and the first one's code in
+ * *first_code ((source file id << 16) | line; 0 when none), and clears them.
+ * In a normal build: BSQ_ERR_UNSUPPORTED, with *count = *first_code = 0. */
+bsq_status bsq_debug_counters(uint32_t* count, uint32_t* first_code);
+
 /* ---------------------------------------------------------------- NVFP4 --
  * nvfp4 page, quantize_nvfp4: along the last dim (K % 16 == 0, else
  * BSQ_ERR_INVALID_ARG -- the page's _check_last_dim), ModelOpt convention

@@ -162,3 +162,19 @@ def test_grouped_mm_host_checks(lib):
     assert g(*args(MX, FWD, 4, 256, 256, 256, err=None)) == INVALID  # the error word is required
     assert g(*args(NV, FWD, 4, 256, 256, 256, rs=None)) == INVALID  # NVFP4 needs its row scales
     assert g(*args(MX, FWD, 4, 0, 256, 256)) == 0  # no tokens: nothing to do
+
+
+def test_debug_counters_in_the_normal_build(lib):
+    """The index-check counters exist only in the bounds-checking build; the
+    normal library answers that it is not one (no CUDA call is made)."""
+    c, f = ctypes.c_uint32(7), ctypes.c_uint32(7)
+    lib.bsq_debug_counters.restype = ctypes.c_int
+    assert lib.bsq_debug_counters(ctypes.byref(c), ctypes.byref(f)) == UNSUPPORTED
+    assert c.value == 0 and f.value == 0
+
+
+def test_debug_build_exports_the_same_symbols():
+    from fp8_microscaling_quantization_b200 import build
+    dbg = ctypes.CDLL(build.build(debug=True))
+    missing = [n for n in declared_entry_points() if not hasattr(dbg, n)]
+    assert not missing, missing
