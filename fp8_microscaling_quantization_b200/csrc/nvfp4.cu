@@ -180,6 +180,11 @@ __global__ void __launch_bounds__(kThreads) nv_flat_quant_kernel(const T* __rest
 // MODE 2 the row's own amax / 2688.  NT is the launch's maximum thread count,
 // MINB the CTAs per SM the register budget is sized for.
 constexpr int kStgMaxThreads = 512, kStgMaxBpt = 4;
+// blocks per thread the launch plan aims for (at most kStgMaxBpt)
+#ifndef BSQ_STG_BPT
+#define BSQ_STG_BPT 4
+#endif
+static_assert(BSQ_STG_BPT >= 1 && BSQ_STG_BPT <= kStgMaxBpt, "blocks per thread of the staged kernel");
 
 template <typename T, int MODE, int S, int NT, int MINB>
 __global__ void __launch_bounds__(NT, MINB)
@@ -324,7 +329,7 @@ static StagedPlan staged_plan(int64_t K) {
     const int64_t stage_bytes = (row_bytes + 127) / 128 * 128;
     // as many blocks per thread as allowed (the per-row work of a thread is
     // shared by more blocks), but at least 64 threads
-    const int bpt = (int)std::max<int64_t>(1, std::min<int64_t>(kStgMaxBpt, bpr / 64));
+    const int bpt = (int)std::max<int64_t>(1, std::min<int64_t>(BSQ_STG_BPT, bpr / 64));
     const int64_t per = (bpr + bpt - 1) / bpt;
     p.nt = (int)((per + 31) / 32 * 32);
     if (p.nt > kStgMaxThreads) return StagedPlan();
