@@ -71,12 +71,12 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "flat": ["flat.cu", "common.cuh", "formats.cuh", "host_util.h"],
-    "nvfp4": ["nvfp4.cu", "common.cuh", "formats.cuh", "host_util.h"],
-    "cache": ["cache.cu", "common.cuh", "formats.cuh", "host_util.h"],
-    "static": ["static.cu", "common.cuh", "formats.cuh", "host_util.h"],
-    "kv": ["kv_cache.cu", "common.cuh", "formats.cuh", "host_util.h"],
-    "gemm": ["grouped_mm.cu", "tcgen05.cuh", "formats.cuh", "host_util.h"],
+    "flat": ["flat.cu", "common.cuh", "formats.cuh", "host_util.h", "debug.cuh"],
+    "nvfp4": ["nvfp4.cu", "common.cuh", "formats.cuh", "host_util.h", "debug.cuh"],
+    "cache": ["cache.cu", "common.cuh", "formats.cuh", "host_util.h", "debug.cuh"],
+    "static": ["static.cu", "common.cuh", "formats.cuh", "host_util.h", "debug.cuh"],
+    "kv": ["kv_cache.cu", "common.cuh", "formats.cuh", "host_util.h", "debug.cuh"],
+    "gemm": ["grouped_mm.cu", "tcgen05.cuh", "formats.cuh", "host_util.h", "debug.cuh"],
 }
 
 
