@@ -37,8 +37,9 @@ def edge_bf16_values():
 # ---------------------------------------------------------------- NVFP4 -----
 
 # Rows of up to 2048 blocks (bf16 K <= 32768) are staged whole in shared
-# memory by bulk copies (at most 4 blocks per thread: K = 8240 gives 515
-# blocks on 288 threads); longer rows up to K = 65536 run the one-CTA-per-row
+# memory by per-thread cp.async copies (at most 4 blocks per thread: K = 8240
+# gives 515 blocks on 160 threads, the last ones with fewer than 4); longer
+# rows up to K = 65536 run the one-CTA-per-row
 # kernel that re-reads the row from L2; K > 65536 takes the two-kernel form
 # (row amax pass, then the flat quantize reading the computed row scales).
 @pytest.mark.parametrize("rows,K", [(256, 2048), (37, 272), (5, 16), (129, 4096), (7, 8240), (3, 40000),
