@@ -103,24 +103,36 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
 template <int FMT, int L>
 __device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg, const NvTables* tab, float out[8]) {
     const float amax_b = group_max<L>(amax8(v));
+    const float2 zero2 = make_float2(0.0f, 0.0f);
     if (FMT == BSQ_FP8) {
         const float p = pow2_scale_fast(amax_b, kE4M3Max, 1.0f / kE4M3Max);
         const float inv = exp2_int(127 - f32_biased_exp(p));
+        const float2 inv2 = make_float2(inv, inv), p2 = make_float2(p, p);
 #pragma unroll
         for (int j = 0; j < 8; j += 2) {
-            const float2 d = e4m3x2_decode_hw(e4m3x2_encode_hw(v[j] * inv, v[j + 1] * inv));
-            out[j] = d.x * p;
-            out[j + 1] = d.y * p;
+            const float2 q = mul_f32x2(make_float2(v[j], v[j + 1]), inv2);  // exact: inv is a power of two
+            const float2 o = mul_f32x2(e4m3x2_decode_hw(e4m3x2_encode_hw(q.x, q.y)), p2);
+            out[j] = o.x;
+            out[j + 1] = o.y;
         }
     } else if (FMT == BSQ_MXFP4) {
         const float p = pow2_scale_fast(amax_b, kE2M1Max, 1.0f / kE2M1Max);
         const float inv = exp2_int(127 - f32_biased_exp(p));
+        const float2 inv2 = make_float2(inv, inv), p2 = make_float2(p, p);
         float q[8], e[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) q[j] = v[j] * inv;
+        for (int j = 0; j < 8; j += 2) {
+            const float2 t = mul_f32x2(make_float2(v[j], v[j + 1]), inv2);
+            q[j] = t.x;
+            q[j + 1] = t.y;
+        }
         e2m1x8_decode_raw(e2m1x8_encode_hw(q), e);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) out[j] = __fmaf_rn(e[j], p, 0.0f);  // exact product
+        for (int j = 0; j < 8; j += 2) {  // exact product, +0.0 for code 8
+            const float2 o = fma_f32x2(make_float2(e[j], e[j + 1]), p2, zero2);
+            out[j] = o.x;
+            out[j + 1] = o.y;
+        }
     } else {
         if (g == 0.0f) {
 #pragma unroll
@@ -150,8 +162,13 @@ __device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg,
             float e[8];
             e2m1x8_decode_raw(codes, e);
             // (e2m1 * s) is exact, then one rounding by g (+0.0 for code 8)
+            const float2 s2 = make_float2(s, s), g2 = make_float2(g, g);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) out[j] = __fmaf_rn(__fmul_rn(e[j], s), g, 0.0f);
+            for (int j = 0; j < 8; j += 2) {
+                const float2 o = fma_f32x2(mul_f32x2(make_float2(e[j], e[j + 1]), s2), g2, zero2);
+                out[j] = o.x;
+                out[j + 1] = o.y;
+            }
         }
     }
 }
@@ -190,22 +207,44 @@ __global__ void __launch_bounds__(kThreads, 8) cache_flat_kernel(const T* __rest
 // Row-resident fake-quant: S lanes per row, every lane loads its (at most
 // NCH) chunks of the zero-padded row before any arithmetic; NVFP4 reduces
 // the row amax over the S lanes.  Handles partial groups and ragged C.
+// With 16-byte rows (VEC) the first row's words are requested before the
+// per-CTA tables are filled, and (when the double buffer is small) the next
+// row's words before the current row is coded, so a warp's rows do not each
+// wait for a DRAM round trip.
 template <typename T, int FMT, int BLOCK, int S, bool VEC, int NCH>
 __global__ void __launch_bounds__(kThreads) cache_row_kernel(const T* __restrict__ x, T* __restrict__ y,
                                                              int64_t rows, int64_t C) {
     constexpr int L = BLOCK / 8;
     constexpr int RPW = 32 / S;
+    constexpr bool PF = VEC && NCH * sizeof(T) <= 4;  // prefetch the next row (at most 16 registers of words)
     __shared__ NvTables tab;
-    if (FMT == BSQ_NVFP4) {
-        fill_nv_tables(&tab);
-        __syncthreads();
-    }
     const int lane = threadIdx.x & 31;
     const int sl = lane % S;
     const int64_t cpr = ((C + BLOCK - 1) / BLOCK) * L;
     const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
     const int64_t wid = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    for (int64_t r0 = wid * RPW; r0 < rows; r0 += warps * RPW) {
+    const int64_t step = warps * RPW;
+    // the words of this lane's chunks of the row starting at r0 (zeros past
+    // the row, the padding and the last row)
+    auto load_row = [&](Raw8<T>* w, int64_t r0) {
+        const int64_t r = r0 + lane / S;
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            const int64_t c = sl + (int64_t)i * S;
+            if (r < rows && c < cpr && C - c * 8 > 0) w[i].load_cs(x + r * C + c * 8);
+            else w[i].zero();
+        }
+    };
+    Raw8<T> cur[NCH], nxt[NCH];
+    const int64_t first = wid * RPW;
+    if (VEC) load_row(cur, first);
+    if (FMT == BSQ_NVFP4) {
+        fill_nv_tables(&tab);
+        __syncthreads();
+    }
+    for (int64_t r0 = first; r0 < rows; r0 += step) {
+        if (PF && r0 + step < rows) load_row(nxt, r0 + step);
+        if (VEC && !PF && r0 != first) load_row(cur, r0);
         const int64_t r = r0 + lane / S;
         const bool row_ok = r < rows;
         const T* xr = x + (row_ok ? r : 0) * C;
@@ -214,14 +253,17 @@ __global__ void __launch_bounds__(kThreads) cache_row_kernel(const T* __restrict
         float m = 0.0f;
 #pragma unroll
         for (int i = 0; i < NCH; ++i) {
-            const int64_t c = sl + (int64_t)i * S;
-            const int64_t n = C - c * 8;
-            if (row_ok && c < cpr && n > 0) {
-                if (VEC && n >= 8) load8(xr + c * 8, v[i]);
-                else load_n(xr + c * 8, (int)(n < 8 ? n : 8), v[i]);
+            if (VEC) {
+                cur[i].get(v[i]);  // zeros where nothing was loaded
             } else {
+                const int64_t c = sl + (int64_t)i * S;
+                const int64_t n = C - c * 8;
+                if (row_ok && c < cpr && n > 0) {
+                    load_n(xr + c * 8, (int)(n < 8 ? n : 8), v[i]);
+                } else {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) v[i][j] = 0.0f;
+                    for (int j = 0; j < 8; ++j) v[i][j] = 0.0f;
+                }
             }
             m = fmaxf(m, amax8(v[i]));
         }
@@ -243,6 +285,10 @@ __global__ void __launch_bounds__(kThreads) cache_row_kernel(const T* __restrict
                     else store_n(yr + c * 8, (int)(n < 8 ? n : 8), out);
                 }
             }
+        }
+        if (PF) {
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) cur[i] = nxt[i];
         }
     }
 }

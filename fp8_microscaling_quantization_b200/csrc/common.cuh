@@ -313,6 +313,19 @@ __device__ __forceinline__ float2 mul_f32x2(float2 a, float2 b) {
     return d;
 }
 
+// fma of two binary32 pairs at once (packed f32x2 fma of sm_100a; each lane
+// rounds once, exactly as a scalar fma does).
+__device__ __forceinline__ float2 fma_f32x2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 A, B, C, D;\n\t"
+        "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\tmov.b64 C, {%6, %7};\n\t"
+        "fma.rn.f32x2 D, A, B, C;\n\t"
+        "mov.b64 {%0, %1}, D;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
 // Asynchronous 16-byte global -> shared copies (cp.async, L2 only), grouped
 // per thread; a thread waits for its own groups with cp_async_wait.
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -494,6 +507,7 @@ template <typename T> struct Raw8;
 template <> struct Raw8<uint16_t> {
     uint4 r;
     __device__ __forceinline__ void load(const uint16_t* p) { r = *reinterpret_cast<const uint4*>(p); }
+    __device__ __forceinline__ void load_cs(const uint16_t* p) { r = __ldcs(reinterpret_cast<const uint4*>(p)); }
     __device__ __forceinline__ void zero() { r = make_uint4(0u, 0u, 0u, 0u); }
     __device__ __forceinline__ void get(float v[8]) const {
         v[0] = bf16_lo(r.x); v[1] = bf16_hi(r.x); v[2] = bf16_lo(r.y); v[3] = bf16_hi(r.y);
@@ -505,6 +519,10 @@ template <> struct Raw8<float> {
     __device__ __forceinline__ void load(const float* p) {
         a = reinterpret_cast<const float4*>(p)[0];
         b = reinterpret_cast<const float4*>(p)[1];
+    }
+    __device__ __forceinline__ void load_cs(const float* p) {
+        a = __ldcs(reinterpret_cast<const float4*>(p));
+        b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
     }
     __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
     __device__ __forceinline__ void get(float v[8]) const {
