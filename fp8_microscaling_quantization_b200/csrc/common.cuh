@@ -484,6 +484,61 @@ __device__ __forceinline__ bool nv_block_codes_fast(const Raw16<T>& raw, uint32_
     return true;
 }
 
+// ---- bf16 NVFP4 block: the correctly rounded quotient, no brackets --------
+//
+// For bf16 elements the code of every element is the e2m1 rounding of
+// q1 = RN(x/d), d = RN(float(s) * g), computed without a division:
+//   y  = RN(1/d)                      (once per block)
+//   q0 = RN(x * y)
+//   r  = RN(q0 * d - x)               (fma)
+//   q1 = RN(q0 - r * y)               (fma)
+// q1 equals the IEEE quotient RN(x/d) for every bf16 significand and every
+// binary32 significand of d (all 2**30 pairs are checked on the CPU by
+// tests/test_exact_brackets.py), hence for all x and d whose intermediate
+// values stay normal: d in [2**-64, 2**100] and |x| * y <= 2**100 (the block
+// amax bounds every element), checked per block; outside that the caller
+// takes the plain rule.  Elements below 2**-126 * d only ever give code 0,
+// with the sign of x.  The products run on -x and -y, so that x = -0.0 gives
+// q1 = -0.0 (and +0.0 gives +0.0), as the division does.
+__device__ __forceinline__ void neg_half_bf16(uint4 w, float v[8]) {
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(ws[i] * 65536u + 0x80000000u);  // (bits << 16) with the sign bit flipped
+        v[2 * i + 1] = __uint_as_float((ws[i] & 0xFFFF0000u) ^ 0x80000000u);
+    }
+}
+
+// The block's codes (low word: elements 0..7) for the positive scale code s,
+// g != 0 and the block amax amax_b.  False when d or the quotients leave the
+// range above (the caller then takes nv_block_codes_slow).
+__device__ __forceinline__ bool nv_block_codes_bf16(const Raw16<uint16_t>& raw, float amax_b, uint32_t s, float g,
+                                                    uint2* codes) {
+    const float d = __fmul_rn(e4m3x2_decode_hw(s).x, g);
+    if (!(d >= 5.4210109e-20f /* 2**-64 */ && d <= 1.2676506e30f /* 2**100 */)) return false;
+    const float y = __frcp_rn(d);
+    if (!(__fmul_rn(amax_b, y) <= 1.2676506e30f)) return false;
+    const float2 ny = make_float2(-y, -y), d2 = make_float2(d, d);
+    uint32_t c[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        float nx[8], q[8];
+        neg_half_bf16(h ? raw.b : raw.a, nx);
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            const float2 xn = make_float2(nx[j], nx[j + 1]);
+            const float2 q0 = mul_f32x2(xn, ny);      // RN(x * y)
+            const float2 r = fma_f32x2(q0, d2, xn);   // RN(q0 * d - x)
+            const float2 q1 = fma_f32x2(r, ny, q0);   // RN(q0 - r * y)
+            q[j] = q1.x;
+            q[j + 1] = q1.y;
+        }
+        c[h] = e2m1x8_encode_hw(q);
+    }
+    *codes = make_uint2(c[0], c[1]);
+    return true;
+}
+
 // 16 consecutive elements (32-byte aligned for bf16).  Plain (L1-cached)
 // loads: the second half of every line a warp touches is then an L1 hit.
 __device__ __forceinline__ void load16(const uint16_t* p, float v[16]) {

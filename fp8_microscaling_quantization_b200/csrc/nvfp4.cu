@@ -167,15 +167,16 @@ __global__ void __launch_bounds__(kThreads) nv_flat_quant_kernel(const T* __rest
 // reads back only its own blocks, so stages are reused without waiting for
 // the other threads.  A first sweep takes the blocks' amaxes; MODE 2 reduces
 // the row amax across the CTA (the kernel's only per-row barrier; per-warp
-// slots alternate by row parity).  A second sweep forms the codes by the
-// division-free brackets.
-//
-// An element whose brackets disagree is settled in place by an exact fma
-// test (nv_block_codes_fast), no division.  With a scale tied to the data (a
-// row or tensor amax / 2688) a few percent of the blocks hold an element whose
-// quotient lands on an e2m1 rounding boundary (an element with the same
-// significand as the amax, for instance), so that path is kept to a few
-// instructions: it runs on one lane of a warp.
+// slots alternate by row parity).  A second sweep forms the codes without a
+// division:
+//  - bf16 rows: every quotient correctly rounded by one fma correction
+//    (nv_block_codes_bf16), the same work for every element, so the warp
+//    never diverges on the data;
+//  - fp32 rows: the bracket codes, and an element whose brackets disagree
+//    settled in place by an exact fma test (nv_block_codes_fast).  With a
+//    scale tied to the data (a row or tensor amax / 2688) a few percent of
+//    the blocks hold such an element (one with the same significand as the
+//    amax, for instance).
 // MODE 0 takes g from g_in, MODE 1 the tensor scale from the partial maxima,
 // MODE 2 the row's own amax / 2688.  NT is the launch's maximum thread count,
 // MINB the CTAs per SM the register budget is sized for.
@@ -199,8 +200,11 @@ __global__ void __launch_bounds__(NT, MINB)
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
     const int bpr = K / 16;
     const uint32_t stage_bytes = ((uint32_t)K * (uint32_t)sizeof(T) + 127u) & ~127u;
-    fill_inv_e4m3(inv_tab);
-    fill_nv_bounds(bounds);
+    constexpr bool kBf16 = sizeof(T) == 2;  // bf16: correctly rounded quotients; fp32: brackets
+    if (!kBf16) {
+        fill_inv_e4m3(inv_tab);
+        fill_nv_bounds(bounds);
+    }
     float g_t = 0.0f, rg_t = 0.0f;
     if (MODE == 1) {
         float m = 0.0f;
@@ -287,7 +291,10 @@ __global__ void __launch_bounds__(NT, MINB)
                     Raw16<T> raw;
                     raw.load_smem(blk);
                     sb = nv_scale_code(am[j], g, rg);
-                    if (!nv_block_codes_fast<T>(raw, blk, sb, g, rg, inv_tab, bounds, &pk)) redo_self |= 1u << j;
+                    bool ok;
+                    if constexpr (kBf16) ok = nv_block_codes_bf16(raw, am[j], sb, g, &pk);
+                    else ok = nv_block_codes_fast<T>(raw, blk, sb, g, rg, inv_tab, bounds, &pk);
+                    if (!ok) redo_self |= 1u << j;
                 }
                 reinterpret_cast<uint2*>(prow)[b] = pk;
                 srow[b] = (uint8_t)sb;

@@ -13,7 +13,16 @@ same argument applies to t1 = RN(RN(a * RN(1/6)) * RN(1/g)), with brackets
 (1 -+ 2**-20) clamped at 2**-9, when g and 1/g are normal and a is 0 or at
 least 2**-120.
 
-Here both shortcuts run in numpy binary32, which rounds each operation to
+bf16 elements.  The kernels code bf16 elements from the quotient itself,
+corrected once: q1 = RN(q0 - r * RN(1/d)) with q0 = RN(x * RN(1/d)) and the
+fma residual r = RN(q0 * d - x).  q1 is RN(x / d) for every pair of a bf16
+significand and a binary32 significand (checked exhaustively below), so its
+code needs no bracket.
+
+Power-of-two scale.  pow2ceil(a / M) is taken from the brackets of
+RN(a * RN(1/M)); only when they straddle a power of two is the division done.
+
+Here the shortcuts run in numpy binary32, which rounds each operation to
 nearest even and keeps subnormals. Their codes come from the oracle's
 roundings and are compared with the oracle's rounding of the plain
 quotients, on random operands and on operands placed within a few ulps of
@@ -353,3 +362,87 @@ def test_straddle_resolution(oracle, m):
     assert np.array_equal(got, want), f"{(got != want).sum()} straddles resolved wrongly"
     # the codes differ by exactly one magnitude step
     assert np.all(np.abs((clo[ok] & 7).astype(np.int64) - (chi[ok] & 7).astype(np.int64)) == 1)
+
+
+# ---- bf16 elements: the correctly rounded quotient by one fma correction ----
+#
+# For bf16 input the kernels code every element as e2m1(q1) with
+#   y = RN(1/d), q0 = RN(x*y), r = RN(q0*d - x) (fma), q1 = RN(q0 - r*y) (fma)
+# and claim q1 = RN(x/d), the binary32 quotient the oracle divides out.  With
+# d in [2**-64, 2**100] and |x*y| <= 2**100, every step that matters stays
+# normal, so the claim depends only on the significands of x and d: the
+# first test below checks all 128 bf16 significands against all 2**23
+# binary32 significands of d.  Binary64 holds q0*d - x exactly; the last
+# rounding is emulated through binary64, and any value that lands near a
+# binary32 midpoint (where that double rounding could differ from the fma's
+# single one) is redone with exact rationals.
+
+def _corrected_quotient(x, d):
+    """(q1, y): the kernels' corrected quotient for binary32 arrays x, d."""
+    from fractions import Fraction
+    with np.errstate(over="ignore", under="ignore", divide="ignore", invalid="ignore"):
+        y = F(1) / d
+        nx, ny = -x, -y
+        q0 = nx * ny                                                     # RN(x * y)
+        r = (q0.astype(np.float64) * d.astype(np.float64) + nx.astype(np.float64)).astype(F)  # fma, exact sum
+        v = r.astype(np.float64) * ny.astype(np.float64) + q0.astype(np.float64)
+        q1 = v.astype(F)
+        q1d = q1.astype(np.float64)
+        near = np.abs(np.abs(v - q1d) - np.abs(np.spacing(q1).astype(np.float64)) / 2) <= np.abs(v) * 2.0 ** -50
+    for i in np.nonzero(near & np.isfinite(v))[0]:
+        exact = Fraction(float(r[i])) * Fraction(float(ny[i])) + Fraction(float(q0[i]))
+        c = q1[i]
+        cands = [np.nextafter(c, F(-np.inf)), c, np.nextafter(c, F(np.inf))]
+        q1[i] = min(cands, key=lambda t: (abs(Fraction(float(t)) - exact), int(np.float32(t).view(np.uint32)) & 1))
+    # q0*d - x must have been exact in binary64 for the emulation of r
+    return q1, y
+
+
+def test_corrected_quotient_every_bf16_significand():
+    """All 2**30 pairs of a bf16 significand X and a binary32 significand D:
+    the corrected quotient equals the IEEE binary32 quotient X / D."""
+    n = 1 << 23
+    D = (np.arange(n, dtype=np.uint32) + np.uint32(0x3F800000)).view(F)
+    wrong = 0
+    for kx in range(128):
+        X = np.full(n, F(1 + kx / 128))
+        q1, _ = _corrected_quotient(X, D)
+        wrong += int((q1 != X / D).sum())
+    assert wrong == 0, f"{wrong} corrected quotients differ from the division"
+
+
+def test_corrected_quotient_is_needed():
+    """The product alone is not the quotient: RN(x * RN(1/d)) misses RN(x/d)
+    for many significand pairs, so the correction step does real work."""
+    D = (np.arange(1 << 20, dtype=np.uint32) * np.uint32(8) + np.uint32(0x3F800000)).view(F)
+    X = np.full(D.size, F(1 + 77 / 128))
+    assert int(((X * (F(1) / D)) != X / D).sum()) > 10_000
+
+
+def test_corrected_quotient_codes_full_range(oracle):
+    """Real exponents, both signs, signed zeros, subnormal bf16 values and the
+    edges of the range the kernels accept: the e2m1 codes of the corrected
+    quotient equal the codes of the division."""
+    rng = np.random.default_rng(31)
+    n = 400_000
+    # divisors across the accepted range, including its edges
+    d = (F(2.0) ** rng.uniform(-64, 100, n).astype(F) * rng.uniform(1, 2, n).astype(F)).astype(F)
+    d[:4] = [F(2.0 ** -64), F(2.0 ** 100), F(2.0 ** -64) * F(1.5), F(2.0 ** 99) * F(1.75)]
+    # bf16 elements: quotients spread over [2**-40, 2**10) and around every boundary
+    t = (F(2.0) ** rng.uniform(-40, 10, n).astype(F)).astype(F)
+    t[: n // 2] = np.array(E2M1_MIDPOINTS + [6.0, 0.5, 1.0, 3.0], dtype=F)[rng.integers(0, 11, n // 2)] * F(
+        1) + (rng.integers(-3, 4, n // 2) * F(2.0 ** -22)).astype(F)
+    xb = ((t * d).astype(F).view(np.uint32) >> 16) << 16                 # truncate to bf16
+    x = xb.view(F) * np.where(rng.integers(0, 2, n) == 1, F(-1), F(1))
+    keep = np.abs(x) * (F(1) / d) <= F(2.0 ** 100)
+    x, d = x[keep], d[keep]
+    # signed zeros and subnormal bf16 values
+    sub = (np.arange(1, 128, dtype=np.uint32) << 16).view(F)
+    x = np.concatenate([x, [F(0.0), F(-0.0)], sub, -sub]).astype(F)
+    d = np.concatenate([d, np.full(2 + 2 * sub.size, F(3.0e-3))]).astype(F)
+    q1, _ = _corrected_quotient(x, d)
+    with np.errstate(over="ignore", under="ignore"):
+        want = oracle.e2m1_round(x / d)
+    got = oracle.e2m1_round(q1)
+    assert np.array_equal(got, want), f"{(got != want).sum()} codes differ"
+    assert np.signbit(q1[x.size - 2 * sub.size - 1]) and not np.signbit(q1[x.size - 2 * sub.size - 2])
