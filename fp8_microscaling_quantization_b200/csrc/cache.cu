@@ -96,8 +96,9 @@ __global__ void __launch_bounds__(kThreads) cache_kernel(const T* __restrict__ x
 
 // Fake-quant of one 8-element chunk in registers (the block's lanes are
 // adjacent; g is the row scale for NVFP4, rg = nv_recip_or_zero(g)).  The
-// power-of-two scales and the NVFP4 codes are taken without a division (see
-// pow2_scale_fast and nv_block_codes_fast); the dequantized value is one
+// power-of-two scales come from the bits of the block amax (pow2_scale_biased)
+// and the NVFP4 codes from the brackets and the fma settling of straddled
+// elements, all without a division; the dequantized value is one
 // multiply by the positive scale, folded with +0.0 into an fma so that code 8
 // (-0.0 from the hardware decode) gives the table's +0.0.
 template <int FMT, int L>
@@ -105,8 +106,8 @@ __device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg,
     const float amax_b = group_max<L>(amax8(v));
     const float2 zero2 = make_float2(0.0f, 0.0f);
     if (FMT == BSQ_FP8) {
-        const float p = pow2_scale_fast(amax_b, kE4M3Max, 1.0f / kE4M3Max);
-        const float inv = exp2_int(127 - f32_biased_exp(p));
+        const uint32_t pb = pow2_scale_biased<8, 0x600000u>(amax_b);  // 448 = 1.75 * 2**8
+        const float p = __uint_as_float(pb << 23), inv = __uint_as_float((254u - pb) << 23);
         const float2 inv2 = make_float2(inv, inv), p2 = make_float2(p, p);
 #pragma unroll
         for (int j = 0; j < 8; j += 2) {
@@ -116,8 +117,8 @@ __device__ __forceinline__ void cache_chunk(const float v[8], float g, float rg,
             out[j + 1] = o.y;
         }
     } else if (FMT == BSQ_MXFP4) {
-        const float p = pow2_scale_fast(amax_b, kE2M1Max, 1.0f / kE2M1Max);
-        const float inv = exp2_int(127 - f32_biased_exp(p));
+        const uint32_t pb = pow2_scale_biased<2, 0x400000u>(amax_b);  // 6 = 1.5 * 2**2
+        const float p = __uint_as_float(pb << 23), inv = __uint_as_float((254u - pb) << 23);
         const float2 inv2 = make_float2(inv, inv), p2 = make_float2(p, p);
         float q[8], e[8];
 #pragma unroll

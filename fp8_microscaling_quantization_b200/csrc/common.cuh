@@ -19,7 +19,6 @@ constexpr int kThreads = 256;
 constexpr float kE2M1Max = 6.0f;       // nvfp4 page E2M1_MAX
 constexpr float kE4M3Max = 448.0f;     // nvfp4 page E4M3_MAX
 constexpr float kE4M3MinSub = 0.001953125f;  // nvfp4 page E4M3_MIN_SUBNORMAL = 2**-9
-constexpr float kF32MinNormal = 1.17549435e-38f;  // 2**-126
 constexpr float kNvGlobalDiv = 2688.0f;  // 6 * 448
 
 template <typename T> struct Elem;
@@ -118,26 +117,19 @@ __device__ __forceinline__ int mx8_exponent(float amax_b) {
     return max(-127, min(127, e));
 }
 
-// Power-of-two block scale pow2ceil(max(amax / fmt_max, 2**-126)).
-__device__ __forceinline__ float pow2_scale(float amax_b, float fmt_max) {
-    float a = __fdiv_rn(amax_b, fmt_max);
-    if (a < kF32MinNormal) a = kF32MinNormal;
-    return pow2_ceil_normal(a);
-}
-
-// The same without the division: q = RN(a * inv_max) (inv_max = RN(1 /
-// fmt_max)) is within two roundings of a / fmt_max and RN(a / fmt_max) within
-// one, and pow2ceil is monotone, so when the brackets RN(q * (1 -+ 2**-21))
-// have the same power-of-two ceiling, that is the rule's value.  Otherwise (a
-// quotient next to a power of two) or for q < 2**-125, the division.
-__device__ __forceinline__ float pow2_scale_fast(float amax_b, float fmt_max, float inv_max) {
-    const float q = __fmul_rn(amax_b, inv_max);
-    if (q >= 2.3509887e-38f /* 2**-125 */) {
-        const float plo = pow2_ceil_normal(__fmul_rn(q, 0.99999952f));
-        const float phi = pow2_ceil_normal(__fmul_rn(q, 1.00000048f));
-        if (plo == phi) return plo;
-    }
-    return pow2_scale(amax_b, fmt_max);
+// Power-of-two block scale pow2ceil(max(RN(a / M), 2**-126)) for a finite
+// a >= 0 and M = m * 2**K, m = 1.75 (448: K = 8, MM = 0x600000) or m = 1.5
+// (6: K = 2, MM = 0x400000): its biased exponent, exactly, from the bits of a.
+// With a = A * 2**E, A in [1, 2): A / m lies in [1/m, 2/m), which holds no
+// power of two but 1, so RN(a / M) is at most 2**(E - K) when A <= m and
+// above it when A > m (then A / m >= 1 + 2**-23 / m, which rounds up, away
+// from 1).  The floor 2**-126 covers zero, subnormal a and every quotient
+// below it.
+template <int K, uint32_t MM>
+__device__ __forceinline__ uint32_t pow2_scale_biased(float a) {
+    const uint32_t b = __float_as_uint(a);
+    const int pb = (int)(b >> 23) - K + ((b & 0x7FFFFFu) > MM ? 1 : 0);
+    return (uint32_t)max(pb, 1);
 }
 
 // NVFP4 block scale byte: e4m3(max((amax_b / 6) / g, 2**-9)).

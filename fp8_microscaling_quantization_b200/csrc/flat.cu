@@ -71,8 +71,9 @@ __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restric
                     if ((lane % L) == 0 && BSQ_DOK(c / L < nchunks / L)) scales[c / L] = (uint8_t)(e + 127);
                 }
             } else {
-                const float p = pow2_scale(amax_b, kE4M3Max);
-                const float inv = exp2_int(127 - f32_biased_exp(p));  // 1 / p, exact
+                const uint32_t pb = pow2_scale_biased<8, 0x600000u>(amax_b);  // 448 = 1.75 * 2**8
+                const float p = __uint_as_float(pb << 23);
+                const float inv = __uint_as_float((254u - pb) << 23);  // 1 / p, exact
                 uint2 w;
                 w.x = e4m3x2_encode_hw(vu[0] * inv, vu[1] * inv) |
                       (e4m3x2_encode_hw(vu[2] * inv, vu[3] * inv) << 16);
@@ -80,7 +81,7 @@ __global__ void __launch_bounds__(kThreads) flat_quant_kernel(const T* __restric
                       (e4m3x2_encode_hw(vu[6] * inv, vu[7] * inv) << 16);
                 if (c < nchunks) {
                     reinterpret_cast<uint2*>(codes)[c] = w;
-                    if ((lane % L) == 0 && BSQ_DOK(c / L < nchunks / L)) scales[c / L] = (uint8_t)f32_biased_exp(p);
+                    if ((lane % L) == 0 && BSQ_DOK(c / L < nchunks / L)) scales[c / L] = (uint8_t)pb;
                 }
             }
         }
@@ -137,19 +138,24 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __rest
 #pragma unroll
                 for (int i = 0; i < EPI / 2; ++i) {
                     const uint32_t word = (i < 2) ? w0[u] : w1[u];
-                    const float2 d = e4m3x2_decode_hw((word >> (16 * (i & 1))) & 0xFFFFu);
-                    v[2 * i] = d.x * p;
-                    v[2 * i + 1] = d.y * p;
+                    const float2 d = mul_f32x2(e4m3x2_decode_hw((word >> (16 * (i & 1))) & 0xFFFFu), make_float2(p, p));
+                    v[2 * i] = d.x;
+                    v[2 * i + 1] = d.y;
                 }
             } else {
-                const float s = (FMT == FMT_MX) ? e8m0_decode(sc[u]) : e4m3_decode(sc[u]);
+                const float s = (FMT == FMT_MX) ? e8m0_decode(sc[u]) : e4m3x2_decode_hw(sc[u]).x;
                 // e2m1 * s is exact (a power of two for MXFP4, 6 significant
                 // bits for NVFP4); the decode already gives code 8 as +0
                 float e[8];
                 e2m1x8_decode_hw(w0[u], e);  // fp32 output: the first EPI = 4 are used
+                const float2 s2 = make_float2(s, s), g2 = make_float2(gr[u], gr[u]);
 #pragma unroll
-                for (int j = 0; j < EPI; ++j)
-                    v[j] = (FMT == FMT_MX) ? __fmul_rn(e[j], s) : __fmul_rn(__fmul_rn(e[j], s), gr[u]);
+                for (int j = 0; j < EPI; j += 2) {
+                    float2 t = mul_f32x2(make_float2(e[j], e[j + 1]), s2);
+                    if (FMT == FMT_NV) t = mul_f32x2(t, g2);
+                    v[j] = t.x;
+                    v[j + 1] = t.y;
+                }
             }
             TOUT* dst = y + it * EPI;
             if (!BSQ_DOK(it < nitems)) continue;

@@ -42,13 +42,6 @@ __device__ __forceinline__ float exp2_int(int e) {
     return __uint_as_float(1u << (e + 149));
 }
 
-// Round a positive normal binary32 up to a power of two.
-__device__ __forceinline__ float pow2_ceil_normal(float a) {
-    uint32_t b = __float_as_uint(a);
-    if ((b & 0x007FFFFFu) == 0) return a;
-    return __uint_as_float((b & 0x7F800000u) + 0x00800000u);
-}
-
 // ------------------------------------------------------------------ e4m3 --
 
 // Nearest finite e4m3 code, ties to even, saturating at 448 (software; used
@@ -118,21 +111,16 @@ __device__ __forceinline__ uint32_t e2m1x8_encode_hw(const float v[8]) {
 
 // Four bytes of packed e2m1 codes -> eight binary32 values (code 2i + j from
 // nibble j of byte i), by the hardware conversion to f16x2 and f16 -> f32
-// (both exact).  The conversion gives -0.0 for code 8; adding +0.0 turns that
-// into the table's +0.0 and leaves every other value unchanged.
+// (both exact).  The conversion gives -0.0 for code 8, so code 8 is first
+// turned into code 0 on the integer pipe: a nibble keeps its sign bit only
+// when its magnitude bits are nonzero (magnitude + 7 carries into bit 3
+// exactly then, and never out of the nibble).  The result is the table's
+// +0.0 for code 8 and every other value unchanged.
+__device__ __forceinline__ void e2m1x8_decode_raw(uint32_t w, float v[8]);
 __device__ __forceinline__ void e2m1x8_decode_hw(uint32_t w, float v[8]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint32_t h2;
-        asm("{\n\t.reg .b8 t;\n\t"
-            "cvt.u8.u32 t, %1;\n\t"
-            "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
-            : "=r"(h2)
-            : "r"(w >> (8 * i)));
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
-        v[2 * i] = __fadd_rn(f.x, 0.0f);
-        v[2 * i + 1] = __fadd_rn(f.y, 0.0f);
-    }
+    const uint32_t mag = w & 0x77777777u;
+    const uint32_t nonzero = (mag + 0x77777777u) & 0x88888888u;
+    e2m1x8_decode_raw(mag | (w & nonzero), v);
 }
 
 

@@ -261,20 +261,19 @@ def test_scaled_reciprocal_at_the_range_edges(oracle):
     check_elements_scaled(oracle, x, ss, gg)
 
 
-# ---- power-of-two block scale without the division -------------------------
+# ---- the power-of-two scales from the bits of the amax ----------------------
 #
-# The cache fake-quant's scale is pow2ceil(max(RN(a / M), 2**-126)) for
-# M = 448 (fp8) or 6 (mxfp4).  q = RN(a * RN(1/M)) is within two roundings of
-# a / M and RN(a / M) within one, and pow2ceil is monotone, so when the two
-# brackets RN(q * (1 -+ 2**-21)) have the same power-of-two ceiling, that is
-# RN(a / M)'s; the kernels divide only when they differ or q < 2**-125.
+# pow2ceil(max(RN(a / M), 2**-126)) for M = 448 = 1.75 * 2**8 and
+# M = 6 = 1.5 * 2**2: with a = A * 2**E (A in [1, 2)), RN(a / M) is at most
+# 2**(E - K) when A <= m and above it when A > m, so the scale's biased
+# exponent is max(biased(a) - K + [mantissa(a) > mantissa(m)], 1).  The
+# kernels take it from the bits; here it is compared with the oracle's
+# power-of-two ceiling of the IEEE quotient.
 
-def pow2_by_bracket(oracle, a, M):
-    with np.errstate(over="ignore", under="ignore"):
-        q = a * (F(1) / F(M))
-        lo, hi = q * LO21, q * HI21
-    plo, phi = oracle.pow2_ceil(np.maximum(lo, F(2.0 ** -126))), oracle.pow2_ceil(np.maximum(hi, F(2.0 ** -126)))
-    return plo, (plo == phi) & (q >= F(2.0 ** -125))
+def pow2_by_bits(a, K, MM):
+    b = a.view(np.uint32).astype(np.int64)
+    pb = (b >> 23) - K + ((b & 0x7FFFFF) > MM)
+    return (np.maximum(pb, 1).astype(np.uint32) << 23).view(np.float32)
 
 
 def pow2_by_division(oracle, a, M):
@@ -282,24 +281,18 @@ def pow2_by_division(oracle, a, M):
         return oracle.pow2_ceil(np.maximum(a / F(M), F(2.0 ** -126)))
 
 
-@pytest.mark.parametrize("M", [448.0, 6.0])
-def test_pow2_scale_brackets(oracle, M):
-    rng = np.random.default_rng(9 + int(M))
-    # random amaxes over the whole normal range, and amaxes within 64 ulps of
-    # M * 2**k for every k (quotients next to a power of two)
-    a1 = (F(2.0) ** rng.uniform(-110, 127, 1_000_000).astype(np.float32)).astype(np.float32)
-    k = np.arange(-120, 120, dtype=np.float64)
-    a0 = (M * 2.0 ** k).astype(np.float32)
-    d = np.arange(-64, 65, dtype=np.int64)
-    a2 = (a0.view(np.uint32).astype(np.int64)[:, None] + d[None, :]).astype(np.uint32).view(np.float32).ravel()
-    a3 = (F(2.0) ** rng.uniform(-149, -110, 100_000).astype(np.float32)).astype(np.float32)  # tiny: floor
-    a = np.concatenate([a1, a2[np.isfinite(a2) & (a2 > 0)], a3])
-    want = pow2_by_division(oracle, a, M)
-    got, decided = pow2_by_bracket(oracle, a, M)
-    bad = decided & (got != want)
+@pytest.mark.parametrize("M,K,MM", [(448.0, 8, 0x600000), (6.0, 2, 0x400000)])
+def test_pow2_scale_bits(oracle, M, K, MM):
+    """Every binary32 significand at the exponents around 1, the floor and the
+    top of the range, every bf16 value, zero and the subnormals."""
+    sig = np.arange(1 << 23, dtype=np.uint32)
+    parts = [(sig | np.uint32(e << 23)).view(np.float32) for e in (1, 2, 9, 10, 118, 119, 120, 121, 127, 128, 254)]
+    parts.append((np.arange(0x0000, 0x7F80, dtype=np.uint32) << 16).view(np.float32))   # all finite bf16 >= 0
+    parts.append(np.arange(0, 1 << 16, 7, dtype=np.uint32).view(np.float32))             # zero, subnormals
+    a = np.concatenate(parts)
+    got, want = pow2_by_bits(a, K, MM), pow2_by_division(oracle, a, M)
+    bad = got != want
     assert not bad.any(), f"{bad.sum()} power-of-two scales differ; first a={a[bad][0]!r}"
-    assert decided[: a1.size].mean() > 0.999
-    assert not decided.all()  # the quotients next to a power of two do reach the division
 
 
 # ---- resolving a straddled bracket without the division ---------------------
