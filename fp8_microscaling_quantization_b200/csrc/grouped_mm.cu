@@ -603,31 +603,64 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_mm_kernel(const __grid_co
                 if (!wait_bar(&sh.acc_empty[acc], ((tile_iter / P::NACC) & 1) ^ 1, sh, args)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * TN);
-                for (int ks = 0; ks < k_steps; ++ks, ++it) {
-                    const int s = it % P::STAGES;
-                    if (!wait_bar(&sh.full[s], (it / P::STAGES) & 1, sh, args)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t ws = st_base + s * P::kStage;
-                    const uint64_t ad0 = (DIR == BSQ_FWD) ? smem_desc(ws, 16, 1024) : smem_desc(ws, BK * 128, 1024);
-                    const uint64_t bd0 = smem_desc(ws + kWStage, 16, 1024);
-#pragma unroll
-                    for (int k16 = 0; k16 < BK / 16; ++k16) {
-                        // the start address field (bits 0-13) cannot carry: the
-                        // stage lies below 256 KiB of shared memory
-                        const uint64_t ad = ad0 + kAStep * k16, bd = bd0 + kBStep * k16;
-                        const uint32_t accum = (ks | k16) != 0 ? 1u : 0u;
-                        if (CG == 1) {
-                            mma_bf16_ss(d_tmem, ad, bd, idesc0, accum);
-                        } else {
-                            mma_bf16_ss_pair(d_tmem, ad, bd, idesc0, accum);
-                            if (n1) mma_bf16_ss_pair(d_tmem + TN, ad, bd + (P::kXHalf >> 4), idesc1, accum);
+                if (CG == 1) {
+                    for (int ks = 0; ks < k_steps; ++ks, ++it) {
+                        const int s = it % P::STAGES;
+                        if (!wait_bar(&sh.full[s], (it / P::STAGES) & 1, sh, args)) {
+                            ok = false;
+                            break;
                         }
+                        tc_fence_after();
+                        const uint32_t ws = st_base + s * P::kStage;
+                        const uint64_t ad0 =
+                            (DIR == BSQ_FWD) ? smem_desc(ws, 16, 1024) : smem_desc(ws, BK * 128, 1024);
+                        const uint64_t bd0 = smem_desc(ws + kWStage, 16, 1024);
+#pragma unroll
+                        for (int k16 = 0; k16 < BK / 16; ++k16) {
+                            const uint64_t ad = ad0 + kAStep * k16, bd = bd0 + kBStep * k16;
+                            const uint32_t accum = (ks | k16) != 0 ? 1u : 0u;
+                            mma_bf16_ss(d_tmem, ad, bd, idesc0, accum);
+                        }
+                        mma_commit(&sh.empty[s]);
                     }
-                    if (CG == 1) mma_commit(&sh.empty[s]);
-                    else mma_commit_pair_multicast(&sh.empty[s], 0x3);
+                } else {
+                    // Pairs.  The MMA thread's instructions per k-step are on
+                    // the critical path (a partial tile's MMAs finish quickly),
+                    // so they are kept few: the descriptors of stage 0 are split
+                    // into 32-bit halves once, a stage's start address is the
+                    // low half plus s * kStage / 16 (the start address field,
+                    // bits 0-13, cannot carry: the stages lie below 256 KiB of
+                    // shared memory), and the one- or two-MMA choice is made
+                    // once per tile.
+                    const uint64_t a00 =
+                        (DIR == BSQ_FWD) ? smem_desc(st_base, 16, 1024) : smem_desc(st_base, BK * 128, 1024);
+                    const uint64_t b00 = smem_desc(st_base + kWStage, 16, 1024);
+                    const uint32_t a_lo0 = (uint32_t)a00, a_hi = (uint32_t)(a00 >> 32);
+                    const uint32_t b_lo0 = (uint32_t)b00, b_hi = (uint32_t)(b00 >> 32);
+                    const uint32_t d1 = d_tmem + TN, xh = (uint32_t)(P::kXHalf >> 4);
+                    auto kstep = [&](int ks, bool two) -> bool {
+                        const int s = it % P::STAGES;
+                        if (!wait_bar(&sh.full[s], (it / P::STAGES) & 1, sh, args)) return false;
+                        tc_fence_after();
+                        const uint32_t so = (uint32_t)(s * (P::kStage >> 4));
+                        const uint32_t al = a_lo0 + so, bl = b_lo0 + so;
+                        const uint32_t acc0 = ks != 0 ? 1u : 0u;
+#pragma unroll
+                        for (int k16 = 0; k16 < BK / 16; ++k16) {
+                            const uint32_t accum = k16 != 0 ? 1u : acc0;
+                            const uint32_t ak = al + (uint32_t)kAStep * k16, bk = bl + (uint32_t)kBStep * k16;
+                            mma_bf16_ss_pair_lh(d_tmem, ak, a_hi, bk, b_hi, idesc0, accum);
+                            if (two) mma_bf16_ss_pair_lh(d1, ak, a_hi, bk + xh, b_hi, idesc1, accum);
+                        }
+                        mma_commit_pair_multicast(&sh.empty[s], 0x3);
+                        ++it;
+                        return true;
+                    };
+                    if (n1) {
+                        for (int ks = 0; ks < k_steps && ok; ++ks) ok = kstep(ks, true);
+                    } else {
+                        for (int ks = 0; ks < k_steps && ok; ++ks) ok = kstep(ks, false);
+                    }
                 }
                 if (ok) {
                     if (CG == 1) mma_commit(&sh.acc_full[acc]);
