@@ -61,13 +61,31 @@ def parse_args():
 
 
 def load_peaks():
+    """The measured denominators from MEASURED_PEAKS.json, each key falling
+    back to FALLBACK_PEAKS when absent or not a positive number (a value may
+    be a number or an object with a "value")."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
-            p = json.load(f)
-        return p, "measured"
+            raw = json.load(f)
     except Exception:
-        return dict(FALLBACK_PEAKS), "fallback"
+        return dict(FALLBACK_PEAKS, sources={k: "fallback" for k in FALLBACK_PEAKS}), "fallback"
+    peaks, measured = dict(FALLBACK_PEAKS), False
+    sources = {k: "fallback" for k in FALLBACK_PEAKS}
+    for k in FALLBACK_PEAKS:
+        v = raw.get(k) if isinstance(raw, dict) else None
+        if isinstance(v, dict):
+            v = v.get("value")
+        try:
+            v = float(v)
+        except (TypeError, ValueError):
+            continue
+        if v > 0:
+            peaks[k] = v
+            sources[k] = "measured"
+            measured = measured or k == "hbm_gbs"
+    peaks["sources"] = sources
+    return peaks, ("measured" if measured else "fallback")
 
 
 KERNEL_SOURCES = {
@@ -984,7 +1002,7 @@ def bench_gemm(torch, bsq, synth, dev, stream, peaks, peak_kind, variants=None, 
                        "half the tokens, half the experts with 1-16 tokens"
         res["routing_skew_mxfp4_fwd"] = skew
     res["err_word"] = int(err.item())
-    res["peak"] = f"{peak} TFLOP/s bf16 dense ({peak_kind}, burst)"
+    res["peak"] = f"{peak} TFLOP/s bf16 dense ({peaks.get('sources', {}).get('bf16_tflops', peak_kind)}, burst)"
     return res
 
 
