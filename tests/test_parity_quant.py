@@ -153,6 +153,11 @@ def test_nvfp4_given_row_scales(B, S, oracle, rows, K):
     g_in = rng.uniform(1e-6, 1e-4, rows).astype(np.float32)
     g_in[min(5, rows - 1)] = 0.0
     g_in[0] = 1e-9  # block scales saturate at 448: codes of quotients far above 6
+    # d = s * g below 2**-64 and above 2**100: outside the range of the
+    # division-free codes, these blocks take the plain division
+    g_in[1] = 1e-25
+    if rows > 6:
+        g_in[6] = 1e33
     p, s, g = B.bsq_quantize_nvfp4(dev_bf16(x), row_scale_in=dev(g_in))
     op, os_, og = oracle.quantize_nvfp4(x, row_scale=g_in)
     assert_bits_equal(host_bits(g), og, "row scale copy")
