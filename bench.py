@@ -29,6 +29,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import threading
@@ -98,15 +99,21 @@ KERNEL_SOURCES = {
 }
 
 
+_COMMENT = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
+
+
 def kernel_source_hash(family):
-    """Hash of the source files a kernel family is built from (a committed
-    ncu traffic figure is only reported while it matches)."""
+    """Hash of the source files a kernel family is built from, with C/C++
+    comments and whitespace runs left out, so that a documentation edit does
+    not retire a committed ncu traffic figure but any change to the code does
+    (the figure is only reported while the hash matches)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "fp8_microscaling_quantization_b200", "csrc")
     for name in KERNEL_SOURCES[family]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            code = " ".join(_COMMENT.sub(" ", f.read()).split())
+        h.update(name.encode())
+        h.update(code.encode())
     return h.hexdigest()[:16]
 
 

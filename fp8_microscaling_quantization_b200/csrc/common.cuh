@@ -343,13 +343,8 @@ __device__ __noinline__ uint2 nv_block_codes_slow(Raw16<T> raw, float g, uint32_
     return make_uint2(c0, e2m1x8_of_quotient(v, d));
 }
 
-// The division-free part of nv_block_codes below: false when the brackets
-// disagree or r is out of range (the caller then takes the plain rule, away
-// from its hot loop).  g != 0.
-
-// The codes of a block whose brackets disagree (nv_block_codes_fast returned
-// false), bit-exact and still without a division.  blk holds the block's 16
-// elements, s its scale code, rg = nv_recip_or_zero(g).  An element whose two
+// Settling a straddled element (the bracket codes of the fp32 NVFP4 path
+// differ), bit-exact and still without a division.  An element whose two
 // bracket codes differ has exactly one e2m1 rounding boundary b between them
 // (0.25, 0.75, 1.25, 1.75, 2.5, 3.5 or 5; the brackets are far narrower than
 // the gaps), and |x| lies within 2**-20 of b * d, d = RN(float(s) * g), so
@@ -357,8 +352,8 @@ __device__ __noinline__ uint2 nv_block_codes_slow(Raw16<T> raw, float g, uint32_
 // hd half an ulp of the float below b (hu / 2 for b = 0.25, a power of two):
 // RN(|x| / d) > b iff e > hu * d, < b iff e < -hd * d, else it equals b, an
 // e2m1 tie that rounds to the even code.  (b's significand is even, so the
-// roundings of b + hu and b - hd are b itself.)  If r is out of range the
-// plain rule is taken.
+// roundings of b + hu and b - hd are b itself.)
+
 // Element i of a block held in shared memory at saddr, as binary32.
 template <typename T>
 __device__ __forceinline__ float elem_smem(uint32_t saddr, int i);
