@@ -624,8 +624,10 @@ static inline bsq_status check_matrix(const char* fn, const void* x, int64_t row
     if (rows < 0 || K < 0) return fail(BSQ_ERR_INVALID_ARG, "%s: negative size (rows=%lld, K=%lld)", fn, (long long)rows, (long long)K);
     if (K % block != 0)
         return fail(BSQ_ERR_INVALID_ARG, "%s: K=%lld is not a whole number of %d-column blocks", fn, (long long)K, block);
+    // 2**35 elements at most: every kernel's 8-element chunk and 16-block
+    // index then fits in 32 bits (tested before rows * K can overflow)
+    if (K > 0 && rows > ((int64_t(1) << 35) - 1) / K) return fail(BSQ_ERR_UNSUPPORTED, "%s: tensor too large", fn);
     if (rows * K > 0 && x == nullptr) return fail(BSQ_ERR_INVALID_ARG, "%s: null pointer", fn);
-    if (rows * K / 8 >= (int64_t(1) << 32)) return fail(BSQ_ERR_UNSUPPORTED, "%s: tensor too large", fn);
     return BSQ_OK;
 }
 

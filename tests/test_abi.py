@@ -178,3 +178,17 @@ def test_debug_build_exports_the_same_symbols():
     dbg = ctypes.CDLL(build.build(debug=True))
     missing = [n for n in declared_entry_points() if not hasattr(dbg, n)]
     assert not missing, missing
+
+
+def test_tensors_past_the_size_limit_are_rejected(lib):
+    """Up to 2**35 elements per call (every chunk and block index then fits
+    in 32 bits); larger shapes, including ones whose rows * K overflows
+    int64, are rejected before anything is launched."""
+    big = [(I64(1 << 20), I64(1 << 15)),            # exactly 2**35
+           (I64(1 << 40), I64(1 << 40)),            # rows * K overflows int64
+           (I64((1 << 62) // 32), I64(64))]
+    for rows, K in big:
+        assert lib.bsq_quantize_mxfp4(FAKE, 0, rows, K, FAKE, FAKE, None) == UNSUPPORTED
+        assert lib.bsq_quantize_nvfp4(FAKE, 0, rows, K, None, FAKE, FAKE, FAKE, None) == UNSUPPORTED
+        assert lib.bsq_dequantize_nvfp4(FAKE, FAKE, FAKE, rows, K, FAKE, 0, None) == UNSUPPORTED
+        assert "too large" in _err(lib)
