@@ -142,17 +142,28 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __rest
                     v[2 * i] = d.x;
                     v[2 * i + 1] = d.y;
                 }
-            } else {
-                const float s = (FMT == FMT_MX) ? e8m0_decode(sc[u]) : e4m3x2_decode_hw(sc[u]).x;
-                // e2m1 * s is exact (a power of two for MXFP4, 6 significant
-                // bits for NVFP4); the decode already gives code 8 as +0
+            } else if (FMT == FMT_MX) {
+                const float s = e8m0_decode(sc[u]);
+                // e2m1 * s is exact (a power of two); the decode gives code 8 as +0
                 float e[8];
                 e2m1x8_decode_hw(w0[u], e);  // fp32 output: the first EPI = 4 are used
-                const float2 s2 = make_float2(s, s), g2 = make_float2(gr[u], gr[u]);
+                const float2 s2 = make_float2(s, s);
 #pragma unroll
                 for (int j = 0; j < EPI; j += 2) {
-                    float2 t = mul_f32x2(make_float2(e[j], e[j + 1]), s2);
-                    if (FMT == FMT_NV) t = mul_f32x2(t, g2);
+                    const float2 t = mul_f32x2(make_float2(e[j], e[j + 1]), s2);
+                    v[j] = t.x;
+                    v[j + 1] = t.y;
+                }
+            } else {
+                // NVFP4: e2m1 * e4m3 is exact (6 significant bits), taken from
+                // the f16 decodes, then one rounding by the row scale
+                const uint32_t s2 = e4m3_to_f16x2(sc[u]);
+                uint32_t e2[4];
+                e2m1x8_to_f16x2(w0[u], e2);  // fp32 output: the first EPI = 4 are used
+                const float2 g2 = make_float2(gr[u], gr[u]);
+#pragma unroll
+                for (int j = 0; j < EPI; j += 2) {
+                    const float2 t = mul_f32x2(mul_f16_to_f32(e2[j / 2], s2), g2);
                     v[j] = t.x;
                     v[j + 1] = t.y;
                 }

@@ -141,6 +141,48 @@ __device__ __forceinline__ void e2m1x8_decode_raw(uint32_t w, float v[8]) {
     }
 }
 
+// Four bytes of packed e2m1 codes -> four f16x2 words (codes 2i, 2i + 1 in
+// word i), code 8 turned into code 0 first as in e2m1x8_decode_hw.  Every
+// e2m1 value is exact in f16.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t h[4]) {
+    const uint32_t mag = w & 0x77777777u;
+    w = mag | (w & ((mag + 0x77777777u) & 0x88888888u));
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        asm("{\n\t.reg .b8 t;\n\t"
+            "cvt.u8.u32 t, %1;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+            : "=r"(h[i])
+            : "r"(w >> (8 * i)));
+}
+
+// The two f16 values of e2 times the f16 value in the low half of s2, as
+// binary32 (a mixed-precision fma with -0.0 added: the products of an e2m1
+// and an e4m3 value have at most 6 significant bits, so they are exact, and
+// x + -0.0 is x for every x, -0.0 and +0.0 included).
+__device__ __forceinline__ float2 mul_f16_to_f32(uint32_t e2, uint32_t s2) {
+    float2 d;
+    asm("{\n\t.reg .f16 el, eh, s, sh;\n\t"
+        "mov.b32 {el, eh}, %2;\n\tmov.b32 {s, sh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, el, s, 0f80000000;\n\t"
+        "fma.rn.f32.f16 %1, eh, s, 0f80000000;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "r"(e2), "r"(s2));
+    return d;
+}
+
+// e4m3 byte (low byte of c) -> its value as f16 in the low half of an
+// f16x2 word (exact: every e4m3 value, subnormals included, is an f16 normal).
+__device__ __forceinline__ uint32_t e4m3_to_f16x2(uint32_t c) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 t;\n\t"
+        "cvt.u16.u32 t, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(h2)
+        : "r"(c & 0xFFu));
+    return h2;
+}
+
 // e8m0 byte -> 2**(code - 127) as binary32 (code 0 is the subnormal 2**-127,
 // 0xFF is NaN).
 __device__ __forceinline__ float e8m0_decode(uint32_t c) {

@@ -94,12 +94,17 @@ __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const uint8_t* con
         for (int u = 0; u < U; ++u) {
             const uint32_t o = o0 + u * kThreads;
             if (o >= items_per_block) continue;
-            const float s = e4m3_decode(sc[u]);
-            float e[8], v[8];
-            e2m1x8_decode_hw(w[u], e);  // fp32 output: only the first 4 are used
-            // e2m1 * s first (exact), then one rounding by g
+            const uint32_t s2 = e4m3_to_f16x2(sc[u]);
+            uint32_t e2[4];
+            float v[8];
+            e2m1x8_to_f16x2(w[u], e2);  // fp32 output: only the first 4 are used
+            // e2m1 * s first (exact, from the f16 decodes), then one rounding by g
 #pragma unroll
-            for (int i = 0; i < EPI; ++i) v[i] = __fmul_rn(__fmul_rn(e[i], s), g);
+            for (int i = 0; i < EPI; i += 2) {
+                const float2 t = mul_f32x2(mul_f16_to_f32(e2[i / 2], s2), make_float2(g, g));
+                v[i] = t.x;
+                v[i + 1] = t.y;
+            }
             TOUT* dst = yb + (int64_t)o * EPI;
             if (!BSQ_DOK((int64_t)b * units_per_block.d < nunits && o < items_per_block)) continue;
             if (sizeof(TOUT) == 2) {
