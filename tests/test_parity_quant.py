@@ -432,7 +432,7 @@ def test_cache_full_size(B, S, oracle, fmt, block, shape):
 
 @pytest.mark.parametrize("fmt", [0, 1, 2])
 @pytest.mark.parametrize("block", [16, 32])
-@pytest.mark.parametrize("C", [1, 8, 13, 40, 128, 520, 4104])
+@pytest.mark.parametrize("C", [1, 8, 13, 40, 128, 264, 300, 520, 640, 4104])
 def test_cache_shapes(B, S, oracle, fmt, block, C):
     x, _ = S.cache_acts(B=2, T=37, C=C, seed=C * 3 + block + fmt)
     xd = dev_bf16(x)
