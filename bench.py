@@ -793,6 +793,32 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
         torch.cuda.synchronize()
         return t.avg_ms("k")
 
+    def graph_timed(calls, reps=7):
+        """Per-launch ms of `calls` (one launch each) captured into one CUDA
+        graph and replayed: the median over `reps` replays of the replay time
+        over len(calls).  The launches run back to back with no host gap."""
+        for c in calls:  # eager once: fills the library's host-side caches
+            c()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for c in calls:
+                c()
+        graph.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(reps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        del graph
+        times.sort()
+        return times[len(times) // 2] / len(calls)
+
     def rec(ms, nbytes, *traffic_keys):
         r = {"us": round(ms * 1e3, 2), "bytes": nbytes, "GB/s": round(nbytes / ms / 1e6, 1),
              "frac_hbm": round(nbytes / ms / 1e6 / hbm, 4)}
@@ -864,6 +890,7 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
     if want("cache"):
         g = torch.Generator(device=dev)
         g.manual_seed(20260003)
+        l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
         cases = [("fp8_b32_4x8192x512", 0, 32, (4, 8192, 512)), ("mxfp4_b32_4x8192x128", 1, 32, (4, 8192, 128)),
                  ("nvfp4_b16_4x2048x512", 2, 16, (4, 2048, 512)), ("fp8_b32_4x2048x520", 0, 32, (4, 2048, 520)),
                  ("mxfp4_b32_4x2048x520", 1, 32, (4, 2048, 520)), ("nvfp4_b16_4x2048x520", 2, 16, (4, 2048, 520))]
@@ -878,12 +905,30 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
             copy_ms = timed(lambda: y.copy_(x), 30, True)
             res[name]["same_size_copy_us"] = round(copy_ms * 1e3, 2)
             res[name]["frac_of_copy"] = round(copy_ms * 1e3 / res[name]["us"], 4)
+            # throughput of back-to-back launches replayed from a CUDA graph,
+            # cycling over input/output copies that together exceed twice the
+            # L2, so that every launch reads and writes HBM; the same-size copy
+            # the same way
+            ns = max(2, -(-2 * l2_bytes // nb))
+            xs = [x.clone() for _ in range(ns)]
+            ys = [torch.empty_like(x) for _ in range(ns)]
+            n_calls = max(60, ns)
+            g_ms = graph_timed([(lambda i=i: bsq.bsq_quantize_cache(xs[i % ns], fmt, blk, y=ys[i % ns]))
+                                for i in range(n_calls)])
+            gc_ms = graph_timed([(lambda i=i: ys[i % ns].copy_(xs[i % ns])) for i in range(n_calls)])
+            res[name].update({"graph_us": round(g_ms * 1e3, 2), "graph_GB/s": round(nb / g_ms / 1e6, 1),
+                              "graph_frac_hbm": round(nb / g_ms / 1e6 / hbm, 4),
+                              "graph_copy_us": round(gc_ms * 1e3, 2), "graph_frac_of_copy": round(gc_ms / g_ms, 4),
+                              "graph_slots": ns, "graph_launches": n_calls})
+            del xs, ys
         gsrc = torch.randn((4, 8192, 512), generator=g, device=dev).to(torch.bfloat16)
         gdst = torch.empty_like(gsrc)
         res["ste_backward_aliased"] = {"us": 0.0, "bytes": 0, "note": "identity: no launch"}
         res["ste_backward_copy_4x8192x512"] = rec(
             timed(lambda: bsq.bsq_quantize_cache_backward(gsrc, gdst), 30, True), 2 * 2 * gsrc.numel())
-        res["note"] = "L2 flushed before every launch (tensors of 8-34 MB)"
+        res["note"] = ("us: one launch, L2 flushed before it (tensors of 8-34 MB); graph_us: per launch, median "
+                       "of 7 replays of a CUDA graph of graph_launches back-to-back launches cycling over "
+                       "graph_slots input/output copies that total at least twice the L2")
         out["quantize_cache"] = res
 
     linear_rows = ("tensor", "row", "gu", "dq", "static")
