@@ -383,6 +383,13 @@ def oracle_cases():
         make_mx8_codes, lambda t: oracle.dequantize_mxfp8(*t, out_dtype=oracle.BF16), K + K // 32 + 2 * K, E * N,
         split2)
 
+    # the FP8 stored form (power-of-two scale per 32-block) on the same weights
+    cases[("fp8_pow2_expert_weights_8x2048x7168", "quantize")] = OracleCase(
+        make_w, lambda x: oracle.quantize_fp8(x, 32), 2 * K + K + K // 32, E * N)
+    cases[("fp8_pow2_expert_weights_8x2048x7168", "dequantize_bf16")] = OracleCase(
+        make_mx8_codes, lambda t: oracle.dequantize_fp8(t[0], t[1], 32, out_dtype=oracle.BF16), K + K // 32 + 2 * K,
+        E * N, split2)
+
     # KV cache: a "row" is one block of 64 tokens x 8 heads x 128
     bt, hd = 64, 8
     rows_kv = bt * hd
@@ -862,6 +869,14 @@ def run_extra(torch, bsq, synth, dev, stream, peaks, peak_kind, only):
                             2 * n + n + n // 32, "mxfp8_quant"),
             "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_mxfp8(c, s, y=y), 10, False),
                                    n + n // 32 + 2 * n, "mxfp8_dequant_bf16"),
+            "note": "inputs and outputs larger than L2"}
+        # the FP8 stored form (e4m3 codes, power-of-two scale per 32-block) on
+        # the same weights: the same kernels with the power-of-two scale rule
+        out["fp8_pow2_expert_weights_8x2048x7168"] = {
+            "quantize": rec(timed(lambda: bsq.bsq_quantize_fp8(x, 32, codes=c, scales=s), 10, False),
+                            2 * n + n + n // 32),
+            "dequantize_bf16": rec(timed(lambda: bsq.bsq_dequantize_fp8(c, s, 32, y=y), 10, False),
+                                   n + n // 32 + 2 * n),
             "note": "inputs and outputs larger than L2"}
         del x, c, s, y
 
