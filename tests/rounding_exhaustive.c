@@ -1,5 +1,6 @@
-/* Exhaustive check of the oracle's three roundings (test code; it links the
- * oracle's library and calls o_e2m1_round, o_e4m3_round and o_f32_to_bf16).
+/* Exhaustive check of the oracle's roundings (test code; it links the
+ * oracle's library and calls o_e2m1_round, o_e4m3_round, o_f32_to_bf16,
+ * o_floor_log2 and o_pow2_ceil).
  *
  * Every finite binary32 bit pattern x is checked for:
  *   - e2m1: the code's magnitude is a nearest value of |x| among the printed
@@ -16,6 +17,10 @@
  * of the binades [2**-10, 2**9), which hold every rounding decision between
  * two codes, and on every 1024th pattern elsewhere (negatives included).
  * Distances are taken in binary64, exact wherever two codes compete.
+ * On every positive finite pattern a: floor_log2 gives the e with
+ * 2**e <= a < 2**(e+1); on every positive normal, the power-of-two ceiling
+ * is a power of two p with a <= p < 2a (+inf above 2**127, where 2a has no
+ * binary32 power of two).
  *
  * Usage: rounding_exhaustive [threads]; prints one line per rounding with
  * its count of failures and exits 0 when there are none. */
@@ -29,6 +34,8 @@
 int o_e2m1_round(float q);
 int o_e4m3_round(float x);
 uint16_t o_f32_to_bf16(float f);
+int o_floor_log2(float a);
+float o_pow2_ceil(float a);
 
 static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
 static double E4M3_MAG[127];
@@ -54,8 +61,8 @@ static int is_nearest(const double* vals, int n, double m, int k) {
 
 typedef struct {
     int t, nt;
-    uint64_t bad_e2m1, bad_bf16, bad_e4m3, n_e4m3;
-    uint32_t first_e2m1, first_bf16, first_e4m3;
+    uint64_t bad_e2m1, bad_bf16, bad_e4m3, n_e4m3, bad_log2, bad_pow2;
+    uint32_t first_e2m1, first_bf16, first_e4m3, first_log2, first_pow2;
 } Job;
 
 static void note(uint64_t* bad, uint32_t* first, uint32_t b) {
@@ -105,6 +112,19 @@ static void* run(void* arg) {
                 j->n_e4m3++;
                 if (((c4 >> 7) & 1) != neg || !e4m3_ok(m, c4 & 0x7F)) note(&j->bad_e4m3, &j->first_e4m3, b);
             }
+            if (!neg && mag != 0) {
+                const int e = o_floor_log2(x);
+                if (!(ldexp(1.0, e) <= m && m < ldexp(1.0, e + 1))) note(&j->bad_log2, &j->first_log2, b);
+                if (mag >= 0x00800000u) { /* normal */
+                    const float p = o_pow2_ceil(x);
+                    uint32_t pb;
+                    memcpy(&pb, &p, 4);
+                    const int ok = (m > ldexp(1.0, 127)) ? (pb == 0x7F800000u)
+                                                         : ((pb & 0x807FFFFFu) == 0 && pb != 0 && (double)p >= m &&
+                                                            (double)p < 2.0 * m);
+                    if (!ok) note(&j->bad_pow2, &j->first_pow2, b);
+                }
+            }
             if (!neg) { /* ascending values */
                 if ((c2 & 7) < prev2 || r < prevb) note(&j->bad_e2m1, &j->first_e2m1, b);
                 prev2 = c2 & 7;
@@ -135,13 +155,17 @@ int main(int argc, char** argv) {
         jobs[t].nt = nt;
         if (pthread_create(&th[t], NULL, run, &jobs[t]) != 0) return 2;
     }
-    uint64_t be = 0, bb = 0, b4 = 0, n4 = 0;
-    uint32_t fe = 0, fb = 0, f4 = 0;
+    uint64_t be = 0, bb = 0, b4 = 0, n4 = 0, bl = 0, bp = 0;
+    uint32_t fe = 0, fb = 0, f4 = 0, fl = 0, fp = 0;
     for (int t = 0; t < nt; ++t) {
         pthread_join(th[t], NULL);
         if (jobs[t].bad_e2m1 && !be) fe = jobs[t].first_e2m1;
         if (jobs[t].bad_bf16 && !bb) fb = jobs[t].first_bf16;
         if (jobs[t].bad_e4m3 && !b4) f4 = jobs[t].first_e4m3;
+        if (jobs[t].bad_log2 && !bl) fl = jobs[t].first_log2;
+        if (jobs[t].bad_pow2 && !bp) fp = jobs[t].first_pow2;
+        bl += jobs[t].bad_log2;
+        bp += jobs[t].bad_pow2;
         be += jobs[t].bad_e2m1;
         bb += jobs[t].bad_bf16;
         b4 += jobs[t].bad_e4m3;
@@ -150,7 +174,9 @@ int main(int argc, char** argv) {
     printf("e2m1 failures %llu first 0x%08x\n", (unsigned long long)be, fe);
     printf("bf16 failures %llu first 0x%08x\n", (unsigned long long)bb, fb);
     printf("e4m3 failures %llu first 0x%08x checked %llu\n", (unsigned long long)b4, f4, (unsigned long long)n4);
+    printf("floor_log2 failures %llu first 0x%08x\n", (unsigned long long)bl, fl);
+    printf("pow2_ceil failures %llu first 0x%08x\n", (unsigned long long)bp, fp);
     free(jobs);
     free(th);
-    return (be || bb || b4) ? 1 : 0;
+    return (be || bb || b4 || bl || bp) ? 1 : 0;
 }
