@@ -270,29 +270,32 @@ def test_scaled_reciprocal_at_the_range_edges(oracle):
 # kernels take it from the bits; here it is compared with the oracle's
 # power-of-two ceiling of the IEEE quotient.
 
-def pow2_by_bits(a, K, MM):
-    b = a.view(np.uint32).astype(np.int64)
-    pb = (b >> 23) - K + ((b & 0x7FFFFF) > MM)
-    return (np.maximum(pb, 1).astype(np.uint32) << 23).view(np.float32)
+def _run_division_free_checker(oracle, tmp_path):
+    """Build and run tests/division_free_exhaustive.c (multi-threaded C, about
+    10 s on 8 cores): the corrected quotient on all 2**30 pairs of a bf16
+    significand and a binary32 significand, and the power-of-two rule for
+    M = 448 and M = 6 on every non-negative finite binary32, against the
+    oracle's power-of-two ceiling of the IEEE quotient."""
+    import os
+    import subprocess
+    lib = oracle.build()
+    exe = str(tmp_path / "division_free_exhaustive")
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-Wall", "-pthread", "-o", exe,
+                           os.path.join(os.path.dirname(os.path.abspath(__file__)), "division_free_exhaustive.c"),
+                           lib, "-Wl,-rpath," + os.path.dirname(lib), "-lm"])
+    r = subprocess.run([exe, str(max(1, len(os.sched_getaffinity(0))))], capture_output=True, text=True,
+                       timeout=3600)
+    return r.returncode, r.stdout + r.stderr
 
 
-def pow2_by_division(oracle, a, M):
-    with np.errstate(under="ignore"):
-        return oracle.pow2_ceil(np.maximum(a / F(M), F(2.0 ** -126)))
-
-
-@pytest.mark.parametrize("M,K,MM", [(448.0, 8, 0x600000), (6.0, 2, 0x400000)])
-def test_pow2_scale_bits(oracle, M, K, MM):
-    """Every binary32 significand at the exponents around 1, the floor and the
-    top of the range, every bf16 value, zero and the subnormals."""
-    sig = np.arange(1 << 23, dtype=np.uint32)
-    parts = [(sig | np.uint32(e << 23)).view(np.float32) for e in (1, 2, 9, 10, 118, 119, 120, 121, 127, 128, 254)]
-    parts.append((np.arange(0x0000, 0x7F80, dtype=np.uint32) << 16).view(np.float32))   # all finite bf16 >= 0
-    parts.append(np.arange(0, 1 << 16, 7, dtype=np.uint32).view(np.float32))             # zero, subnormals
-    a = np.concatenate(parts)
-    got, want = pow2_by_bits(a, K, MM), pow2_by_division(oracle, a, M)
-    bad = got != want
-    assert not bad.any(), f"{bad.sum()} power-of-two scales differ; first a={a[bad][0]!r}"
+def test_pow2_scale_bits_and_corrected_quotient_exhaustive(oracle, tmp_path):
+    """The power-of-two scale from the bits of the amax, for M = 448 and
+    M = 6, on every non-negative finite binary32; and every corrected
+    quotient of a bf16 significand by a binary32 significand."""
+    rc, out = _run_division_free_checker(oracle, tmp_path)
+    assert rc == 0, out
+    for what in ("corrected_quotient", "pow2_448", "pow2_6"):
+        assert f"{what} failures 0 " in out, out
 
 
 # ---- resolving a straddled bracket without the division ---------------------
@@ -389,19 +392,6 @@ def _corrected_quotient(x, d):
         q1[i] = min(cands, key=lambda t: (abs(Fraction(float(t)) - exact), int(np.float32(t).view(np.uint32)) & 1))
     # q0*d - x must have been exact in binary64 for the emulation of r
     return q1, y
-
-
-def test_corrected_quotient_every_bf16_significand():
-    """All 2**30 pairs of a bf16 significand X and a binary32 significand D:
-    the corrected quotient equals the IEEE binary32 quotient X / D."""
-    n = 1 << 23
-    D = (np.arange(n, dtype=np.uint32) + np.uint32(0x3F800000)).view(F)
-    wrong = 0
-    for kx in range(128):
-        X = np.full(n, F(1 + kx / 128))
-        q1, _ = _corrected_quotient(X, D)
-        wrong += int((q1 != X / D).sum())
-    assert wrong == 0, f"{wrong} corrected quotients differ from the division"
 
 
 def test_corrected_quotient_is_needed():
