@@ -23,8 +23,11 @@
  *     data between calls (the one exception, the file-scope scratch of
  *     bsq_quantize_nvfp4_tensor_noalloc, is described there); it caches only
  *     host-side facts (SM count, occupancy, the tensor-map encoder).  Outputs
- *     are written in place, so buffer addresses stay stable (CUDA graph
- *     friendly).  Inputs are never modified, except that
+ *     are written in place, so buffer addresses stay stable.  Once an entry
+ *     point has run on a device outside any stream capture (which fills
+ *     those host-side caches), its later calls may be captured into a CUDA
+ *     graph on the caller's stream and replayed.  Inputs are never
+ *     modified, except that
  *     bsq_fake_quantize_nvfp4_static may be asked to write over its input.
  *   - Work is enqueued on `stream` and is asynchronous.  Only argument
  *     validation runs on the host; a rejected call launches nothing.
